@@ -1,0 +1,123 @@
+"""fp64 CPU oracle for the mHC pre and post stages (ctypes wrapper around mhc_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  The tests, the package smoke check and the benchmark's
+CPU-baseline / reference leg may import this module; the product path never does and
+has no CPU fallback.  It shares no code with the CUDA library.
+
+What each function follows (page title, section / equation):
+  * sinkhorn  -- "DeepSeek-V4/mhc" page, equations sinkhorn-init and sinkhorn;
+                 slavadubrov.com mHC article, section "Sinkhorn-Knopp-projectie".
+  * mhc_pre   -- "DeepSeek-V4/mhc" page, "动态参数化怎么实现": equations rmsnorm,
+                 a/b/c-tilde and gate; slavadubrov.com article Eq. 3 (read map).
+  * mhc_post  -- slavadubrov.com article, "Kernmechanismen" Eq. 3; the knowledge
+                 page's HC update equation.
+
+Parity pins for every function live in tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mhc_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile mhc_oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_sinkhorn.argtypes = [_dp, ctypes.c_int, ctypes.c_int, _dp]
+            lib.oracle_sinkhorn.restype = None
+            lib.oracle_mhc_pre.argtypes = [_dp, _dp, _dp, _dp, _dp,
+                                           ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                           ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_double, ctypes.c_int, _dp, _dp, ctypes.c_int]
+            lib.oracle_mhc_pre.restype = None
+            lib.oracle_mhc_post.argtypes = [_dp, _dp, _dp, ctypes.c_long, ctypes.c_int,
+                                            ctypes.c_int, _dp, ctypes.c_int]
+            lib.oracle_mhc_post.restype = None
+            lib.oracle_threads_used.argtypes = [ctypes.c_int]
+            lib.oracle_threads_used.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _c(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_dp)
+
+
+def sinkhorn(logits, t_max: int = 20) -> np.ndarray:
+    """exp(logits), then t_max rounds of column- then row-normalisation (n x n)."""
+    L = _c(logits)
+    n = L.shape[0]
+    assert L.shape == (n, n)
+    out = np.empty_like(L)
+    _load().oracle_sinkhorn(_p(L), n, int(t_max), _p(out))
+    return out
+
+
+def mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+            eps: float = 1e-20, t_max: int = 20, nthreads: int = 1):
+    """Pre stage.  X [T, n, d] -> (x_in [T, d], H [T, n*n+2n]) in fp64."""
+    X = _c(X)
+    T, n, d = X.shape
+    m = n * n + 2 * n
+    phi = _c(phi)
+    assert phi.shape == (n * d, m), phi.shape
+    b_pre, b_post, b_res = _c(b_pre).reshape(n), _c(b_post).reshape(n), _c(b_res).reshape(n * n)
+    x_in = np.empty((T, d), np.float64)
+    H = np.empty((T, m), np.float64)
+    _load().oracle_mhc_pre(_p(X), _p(phi), _p(b_pre), _p(b_post), _p(b_res),
+                           float(alpha_pre), float(alpha_post), float(alpha_res),
+                           T, n, d, float(eps), int(t_max), _p(x_in), _p(H), int(nthreads))
+    return x_in, H
+
+
+def mhc_post(X, F_out, H, nthreads: int = 1) -> np.ndarray:
+    """Post stage.  X [T, n, d], F_out [T, d], H [T, m] -> X' [T, n, d] in fp64."""
+    X, F_out, H = _c(X), _c(F_out), _c(H)
+    T, n, d = X.shape
+    assert F_out.shape == (T, d) and H.shape == (T, n * n + 2 * n)
+    out = np.empty_like(X)
+    _load().oracle_mhc_post(_p(X), _p(F_out), _p(H), T, n, d, _p(out), int(nthreads))
+    return out
+
+
+def threads_used(nthreads: int) -> int:
+    """How many OpenMP threads a request of `nthreads` actually gets."""
+    return int(_load().oracle_threads_used(int(nthreads)))
+
+
+def split_H(H: np.ndarray, n: int):
+    """Split coefficient rows [.., m] into (H_pre [..,n], H_res [..,n,n], H_post [..,n])."""
+    H = np.asarray(H)
+    lead = H.shape[:-1]
+    return (H[..., :n], H[..., n:n + n * n].reshape(*lead, n, n), H[..., n + n * n:])
