@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the mHC forward hot path (pre + post) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...        (one process per GPU)
+
+One step = mhc_pre + mhc_post over one batch of T tokens (the whole hot path; F_out is a
+given input, the sub-layer F itself is not part of the path).  Default workload: T = 16384
+tokens (4 x 4096), n = 4 streams, d = 4096, bf16 storage, fp32 arithmetic, 1 % outlier
+channels; inputs are synthetic and seeded (mhc_hyper_connections_b200.workloads).  The
+workload's inputs (X 512 MiB + F_out 128 MiB) are larger than L2, so no L2 flush is
+needed between steps.
+
+Multi-GPU: tokens are independent, so every rank runs its own T-token batch (weak
+scaling, no data-path collective); the time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle instead, on
+the host cores, over a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "mHC pre+post tokens/s and achieved HBM GB/s (% of roofline), n=4 d=4096 bf16"
+NOMINAL_HBM_GBS = 8000.0          # the target's roofline denominator ("~8 TB/s")
+FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
+
+# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum) for
+# the named kernel on the headline workload, with the sha256 of the kernel source it was
+# measured on; reported as null once that source changes.
+NCU_TRAFFIC = {}
+
+
+def _hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def _src_sha(rel):
+    try:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            return hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+
+
+def bytes_per_token(n, d, es):
+    """Algorithmic HBM bytes per token.  pre: reads X (n d), writes x_in (d) and H (m fp32);
+    post: reads X (n d), F_out (d), H_res + H_post ((n^2 + n) fp32), writes X' (n d)."""
+    m = n * n + 2 * n
+    pre = (n + 1) * d * es + 4 * m
+    post = (2 * n + 1) * d * es + 4 * (n * n + n)
+    return pre, post
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons, n_all = [], None, set(), 0
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            n_all += 1
+            if not (t0 - 0.05 <= ts <= t1 + 0.15):
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                    "samples": 0, "note": "no nvidia-smi sample fell inside the timed region"}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm (oracle)
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from mhc_hyper_connections_b200 import workloads as wl
+
+    w = wl.make_config(args.config)
+    cores = os.cpu_count() or 1
+    used = oracle.threads_used(cores)
+    s = w.scalars()
+
+    def step(sub):
+        X = sub.values(sub.X)
+        F = sub.values(sub.F_out)
+        t0 = time.perf_counter()
+        _, H = oracle.mhc_pre(X, sub.phi, sub.b_pre, sub.b_post, sub.b_res, s["alpha_pre"],
+                              s["alpha_post"], s["alpha_res"], eps=s["eps"], t_max=s["t_max"],
+                              nthreads=cores)
+        oracle.mhc_post(X, F, H, nthreads=cores)
+        return time.perf_counter() - t0
+
+    # size the per-step sample so the whole run stays within ~2 minutes
+    cal = max(step(w.tokens(np.arange(min(64, w.T)))) / min(64, w.T), 1e-7)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    per_step = int(max(1, min(w.T, budget / cal)))
+    rng = np.random.default_rng(0)
+    subs = [w.tokens(np.sort(rng.choice(w.T, per_step, replace=False))) for _ in range(4)]
+    for k in range(args.warmup):
+        step(subs[k % 4])
+    tot = 0.0
+    for k in range(args.steps):
+        tot += step(subs[k % 4])
+    value = per_step * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "T": w.T, "n": w.n, "d": w.d,
+                   "storage": w.dtype, "tokens_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                         "sample": f"{per_step} random tokens of the {w.T}-token batch per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(w, seconds=10.0, cap=4096):
+    """The oracle as it stands, on the host cores, over a bounded token sample."""
+    import numpy as np
+
+    import oracle
+    cores = os.cpu_count() or 1
+    used = oracle.threads_used(cores)
+    s = w.scalars()
+
+    def run(sub):
+        X = sub.values(sub.X)
+        F = sub.values(sub.F_out)
+        t0 = time.perf_counter()
+        _, H = oracle.mhc_pre(X, sub.phi, sub.b_pre, sub.b_post, sub.b_res, s["alpha_pre"],
+                              s["alpha_post"], s["alpha_res"], eps=s["eps"], t_max=s["t_max"],
+                              nthreads=cores)
+        oracle.mhc_post(X, F, H, nthreads=cores)
+        return time.perf_counter() - t0
+
+    k0 = min(64, w.T)
+    per_tok = max(run(w.tokens(np.arange(k0))) / k0, 1e-7)
+    ns = int(max(k0, min(w.T, cap, seconds / per_tok)))
+    idx = np.sort(np.random.default_rng(7).choice(w.T, ns, replace=False))
+    dt = run(w.tokens(idx))
+    return {"value": ns / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{ns} random tokens of the {w.T}-token batch ({dt:.1f} s, fp64, "
+                      f"{used} OpenMP threads)"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import mhc_hyper_connections_b200 as mhc
+    from mhc_hyper_connections_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = wl.make_config(args.config)
+    T, n, d = w.T, w.n, w.d
+    es = 2 if w.dtype == "bf16" else 4
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    X, F = to_dev(w.X), to_dev(w.F_out)
+    phi, b_pre, b_post, b_res = (to_dev(a) for a in (w.phi, w.b_pre, w.b_post, w.b_res))
+    x_in = torch.empty(T, d, dtype=tdt, device=dev)
+    H = torch.empty(T, w.m, dtype=torch.float32, device=dev)
+    Y = torch.empty_like(X)
+    s = w.scalars()
+    path = mhc.mhc_pre_path_for(T, n, d, tdt)
+
+    def pre():
+        mhc.mhc_pre(X, phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
+                    s["alpha_res"], s["eps"], s["t_max"], x_in, H)
+
+    def post():
+        mhc.mhc_post(X, F, H, Y)
+
+    for _ in range(args.warmup):
+        pre()
+        post()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps, events on the launching (current) stream
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local_rank)
+    clk.start()
+    time.sleep(0.6)                       # let nvidia-smi start sampling
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record()
+    for k in range(K):
+        e = evs[k]
+        e[0].record()
+        pre()
+        e[1].record()
+        post()
+        e[2].record()
+    end.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    time.sleep(0.3)
+    clk.stop()
+    ms_total = max_over_ranks(start.elapsed_time(end))
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    post_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    clocks = clk.summary(t_wall0, t_wall1)
+
+    value = world * T * K / (ms_total / 1e3)
+    peak, peak_src = _hbm_peak()
+    b_pre, b_post = bytes_per_token(n, d, es)
+    kern = {"pre": {"ms": pre_ms, "bytes_per_launch": b_pre * T,
+                    "gbs": b_pre * T / (pre_ms / 1e3) / 1e9,
+                    "path": {1: "generic", 2: "cluster_tc"}.get(path, str(path)),
+                    "source": "mhc_hyper_connections_b200/csrc/" +
+                              ("pre_cluster_tc.cu" if path == 2 else "pre_generic.cu")},
+            "post": {"ms": post_ms, "bytes_per_launch": b_post * T,
+                     "gbs": b_post * T / (post_ms / 1e3) / 1e9,
+                     "source": "mhc_hyper_connections_b200/csrc/post.cu"}}
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    traffic = None
+    rec = NCU_TRAFFIC.get((dom, args.config))
+    if rec and rec[1] == _src_sha(kern[dom]["source"]):
+        traffic = rec[0]
+    achieved = kern[dom]["gbs"]
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": kern[dom]["bytes_per_launch"]}
+    b_dep = b_pre + b_post
+    step_gbs = b_dep * T * world / (ms_total / 1e3 / K) / 1e9 / world
+    hbm = {"B_dep_bytes_per_token": b_dep, "B_lit_bytes_per_token": (2 * n + 2) * d * es,
+           "gbs_per_gpu": step_gbs, "frac_of_8TBs": step_gbs / NOMINAL_HBM_GBS,
+           "frac_of_measured": step_gbs / peak,
+           "frac_of_8TBs_lit": (2 * n + 2) * d * es * T / (ms_total / 1e3 / K) / 1e9 / NOMINAL_HBM_GBS}
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(1, min(K, args.e2e_steps))
+        Xh = torch.empty_like(X, device="cpu").pin_memory()
+        Fh = torch.empty_like(F, device="cpu").pin_memory()
+        Xh.copy_(X)
+        Fh.copy_(F)
+        xo = torch.empty_like(x_in, device="cpu").pin_memory()
+        Ho = torch.empty_like(H, device="cpu").pin_memory()
+        Yo = torch.empty_like(Y, device="cpu").pin_memory()
+
+        def e2e_step():
+            X.copy_(Xh, non_blocking=True)
+            F.copy_(Fh, non_blocking=True)
+            pre()
+            post()
+            xo.copy_(x_in, non_blocking=True)
+            Ho.copy_(H, non_blocking=True)
+            Yo.copy_(Y, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(Ke):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b))
+        barrier()
+        e2e = {"value": world * T * Ke / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": (X.numel() + F.numel()) * es,
+               "d2h_bytes_per_step": (x_in.numel() * es + H.numel() * 4 + Y.numel() * es),
+               "steps": Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, seconds=args.cpu_seconds)
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_total / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": args.config, "T": T, "n": n, "d": d, "tokens_per_gpu": T,
+                   "parallelism": f"replicas x{world} (token shards, no collective)",
+                   "l2": "inputs larger than L2 (X 512 MiB + F_out 128 MiB), no flush",
+                   "alpha": s["alpha_pre"], "t_max": s["t_max"], "eps": s["eps"]},
+        "roofline": roofline, "hbm": hbm, "kernels": kern, "clocks": clocks, "e2e": e2e,
+        "cpu_baseline": cpu, "gpu_launches": 2 * K,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    from mhc_hyper_connections_b200 import workloads as wl
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=wl.HEADLINE, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 needs one process per GPU (torchrun --nproc-per-node N)")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

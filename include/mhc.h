@@ -1,0 +1,142 @@
+/*
+ * mhc.h -- C ABI of the B200 (sm_100a) mHC forward hot path.
+ *
+ * mHC (Manifold-Constrained Hyper-Connections) keeps n residual streams per token,
+ * X_t in R^{n x d}, and wraps every sub-layer F in two per-token stages:
+ *
+ *   pre   x_hat = RMSNorm(vec X_t)   h = x_hat . phi   (logits, gates, Sinkhorn)
+ *         x_in  = H_pre X_t                      -> fed to the sub-layer F
+ *   post  X'_t  = H_res X_t + H_post^T F_out_t    -> the next layer's residual
+ *
+ * Sources ("page" = the web page of that title):
+ *   - "DeepSeek-V4/mhc" knowledge page, section "动态参数化怎么实现": equations
+ *     rmsnorm, a-tilde, b-tilde, c-tilde (logits), gate (sigmoid / 2 sigmoid),
+ *     sinkhorn-init and sinkhorn (t_max = 20); its mixed-precision table (phi GEMM
+ *     at TF32 or better, X in bf16, RMSNorm and Sinkhorn in fp32); its I/O-cost
+ *     table (the n^2 + 2n coefficients per token handed from pre to post).
+ *   - "DeepSeek mHC: Manifold-Constrained Hyper-Connections" (slavadubrov.com),
+ *     section "Kernmechanismen", Eq. 3: x_{l+1} = H_res x_l + H_post^T F(H_pre x_l);
+ *     section "Details van de parameterisatie": H_pre in (0,1), H_post in (0,2).
+ *
+ * Conventions shared by every entry point
+ *   - All data pointers are DEVICE pointers.  The caller allocates and owns every
+ *     buffer; the library allocates no device memory and keeps no state between
+ *     calls except a per-device cache of kernel launch limits.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Arguments are validated on the host before any launch; a rejected
+ *     call launches nothing and returns a non-zero mhc_status.  MHC_ERR_CUDA means
+ *     a launch failed; mhc_last_error() then describes it (per host thread).
+ *   - Layouts are contiguous row-major:
+ *       X, X_out   [T, n, d]   stream i of token t at X + (t*n + i)*d
+ *       F_out, x_in[T, d]
+ *       phi        [n*d, m]    fp32, row k = i*d + c (the row-stacked flatten of X_t),
+ *                              columns [pre (n) | res (n*n, row-major) | post (n)]
+ *       H          [T, m]      fp32, m = n*n + 2n, per token [H_pre | H_res | H_post],
+ *                              H_res row-major: H_res[i][j] weights input stream j
+ *                              into output stream i.
+ *       b_pre [n], b_post [n], b_res [n*n] (row-major), all fp32.
+ *   - `dt` is the storage type of X, F_out, x_in and X_out; phi, biases and H are
+ *     always fp32.  Arithmetic is fp32 (the projection accumulates in fp32 with phi
+ *     carried at 16 significant bits or more).
+ *   - Limits: 1 <= n <= 8 (a library limit, not the method's), d >= 1, T >= 0,
+ *     0 <= t_max <= 1000.  T == 0 returns MHC_OK and launches nothing.
+ *   - Alignment: every array must be aligned to its element size (else
+ *     MHC_ERR_ALIGN).  16-byte-aligned arrays with d a multiple of 16/sizeof(elem)
+ *     take the vectorised kernels; others take a scalar kernel with the same results
+ *     up to fp32 rounding order.
+ *   - Aliasing: outputs may not overlap any input or each other (MHC_ERR_ALIAS).
+ *   - NaN and Inf propagate; nothing on the hot path checks values.
+ */
+#ifndef MHC_H
+#define MHC_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                        /* = cudaStream_t without the CUDA headers */
+typedef struct CUstream_st* mhc_stream_t;
+
+typedef enum {
+    MHC_OK = 0,
+    MHC_ERR_NULL = 1,          /* a required pointer is NULL (with T > 0)            */
+    MHC_ERR_SHAPE = 2,         /* n, d, T or t_max out of range, or size overflow    */
+    MHC_ERR_ALIGN = 3,         /* a pointer is not aligned to its element size       */
+    MHC_ERR_DTYPE = 4,         /* dt is not an mhc_dtype value                       */
+    MHC_ERR_UNSUPPORTED = 5,   /* the requested kernel path cannot run this problem  */
+    MHC_ERR_CUDA = 6,          /* a CUDA call or launch failed                       */
+    MHC_ERR_ALIAS = 7          /* an output overlaps an input or another output      */
+} mhc_status;
+
+typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
+
+/* Kernel paths of the pre stage (mhc_pre picks MHC_PRE_AUTO). */
+typedef enum {
+    MHC_PRE_AUTO = 0,          /* the fastest path that supports the problem          */
+    MHC_PRE_GENERIC = 1,       /* CUDA-core kernel: any n <= 8, any d, f32 or bf16    */
+    MHC_PRE_CLUSTER_TC = 2     /* thread-block-cluster tensor-core kernel (bf16,      */
+                               /* n <= 4, d in {1024,2048,3072,4096}; see mhc_pre_path)*/
+} mhc_pre_path;
+
+/*
+ * mhc_pre -- the pre stage for T tokens.
+ * Defined by the "DeepSeek-V4/mhc" page equations rmsnorm, a/b/c-tilde, gate,
+ * sinkhorn-init and sinkhorn, and the read map H_pre x_l of the slavadubrov.com Eq. 3:
+ *   r      = sqrt(mean_k v_k^2 + eps)              v = vec(X_t), k = i*d + c
+ *   h      = (v / r) . phi                          [m]
+ *   H_pre  = sigmoid(alpha_pre * h[0:n] + b_pre)
+ *   H_res  = SK_{t_max}(exp(alpha_res * Mat(h[n:n+n^2]) + b_res))
+ *            (each round: divide every column by its sum, then every row by its sum)
+ *   H_post = 2 sigmoid(alpha_post * h[n+n^2:m] + b_post)
+ *   x_in   = sum_i H_pre[i] X_t[i, :]               (raw X, not x_hat)
+ * Inputs : X [T,n,d] (dt), phi [n*d, m], b_pre [n], b_post [n], b_res [n*n],
+ *          alpha_*, eps (the page uses 1e-20), t_max (the page uses 20).
+ * Outputs: x_in [T,d] (dt), H [T,m] (fp32) = [H_pre | H_res | H_post] per token.
+ * Errors : see "Conventions"; MHC_ERR_CUDA if a launch fails.
+ */
+mhc_status mhc_pre(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                   const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                   int64_t T, int n, int d, float eps, int t_max, mhc_dtype dt,
+                   void* x_in, float* H, mhc_stream_t stream);
+
+/*
+ * mhc_pre_with_path -- mhc_pre on an explicitly chosen kernel path (same arguments and
+ * results).  Returns MHC_ERR_UNSUPPORTED, launching nothing, if `path` cannot run the
+ * problem on the current device.
+ */
+mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre,
+                             const float* b_post, const float* b_res, float alpha_pre,
+                             float alpha_post, float alpha_res, int64_t T, int n, int d,
+                             float eps, int t_max, mhc_dtype dt, void* x_in, float* H,
+                             mhc_stream_t stream, mhc_pre_path path);
+
+/*
+ * mhc_pre_path -- the path MHC_PRE_AUTO would take for this problem on the current
+ * device (host-side query; launches nothing).  Returns MHC_PRE_GENERIC or
+ * MHC_PRE_CLUSTER_TC.
+ */
+mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt);
+
+/*
+ * mhc_post -- the post/res merge for T tokens (slavadubrov.com Eq. 3, first and second
+ * term; the "Post-Res fused kernel" row of the knowledge page's kernel table, which
+ * reads X and F_out once):
+ *   X_out[t, i, :] = sum_j H_res[i][j] X[t, j, :] + H_post[i] F_out[t, :]
+ * Inputs : X [T,n,d] (dt), F_out [T,d] (dt), H [T,m] fp32 as written by mhc_pre.
+ * Output : X_out [T,n,d] (dt); may not alias X, F_out or H.
+ */
+mhc_status mhc_post(const void* X, const void* F_out, const float* H, int64_t T, int n, int d,
+                    mhc_dtype dt, void* X_out, mhc_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+const char* mhc_status_string(mhc_status status);
+
+/* Text of the last MHC_ERR_CUDA raised on the calling host thread ("" if none). */
+const char* mhc_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MHC_H */

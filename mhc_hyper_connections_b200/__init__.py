@@ -1,0 +1,185 @@
+"""mhc_hyper_connections_b200 -- B200-native (sm_100a) mHC forward hot path.
+
+Thin Python binding over the C ABI in include/mhc.h (libmhc_b200.so, built in-tree by
+``python -m mhc_hyper_connections_b200.build``).  The functions here only marshal
+arguments: every step of the path runs in the library's CUDA kernels, and there is no
+CPU fallback -- if the library is missing the calls raise.
+
+    mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
+            x_in, H)                -> writes x_in [T, d] and H [T, n*n+2n]
+    mhc_post(X, F_out, H, X_out)    -> writes X_out [T, n, d]
+
+Tensors are torch CUDA tensors (contiguous; X/F_out/x_in/X_out bf16 or fp32, phi, biases
+and H fp32).  Calls are asynchronous on the current torch stream unless ``stream`` (a
+torch.cuda.Stream or a raw cudaStream_t integer) is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_post", "mhc_pre_path_for", "MhcError",
+           "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
+           "load_library", "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmhc_b200.so")
+
+MHC_F32, MHC_BF16 = 0, 1
+PRE_AUTO, PRE_GENERIC, PRE_CLUSTER_TC = 0, 1, 2
+_STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN",
+           4: "MHC_ERR_DTYPE", 5: "MHC_ERR_UNSUPPORTED", 6: "MHC_ERR_CUDA", 7: "MHC_ERR_ALIAS"}
+
+# Every function include/mhc.h declares.
+EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_path_for", "mhc_post",
+                    "mhc_status_string", "mhc_last_error")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MhcError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        self.name = _STATUS.get(status, str(status))
+        super().__init__(f"{where}: {self.name}" + (f" ({detail})" if detail else ""))
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libmhc_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library {_LIB_PATH} is missing: build it with "
+                               "`python -m mhc_hyper_connections_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, fp, i64, ci, cf = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                               ctypes.c_float)
+        pre_args = [vp, fp, fp, fp, fp, cf, cf, cf, i64, ci, ci, cf, ci, ci, vp, fp, vp]
+        lib.mhc_pre.argtypes = pre_args
+        lib.mhc_pre.restype = ci
+        lib.mhc_pre_with_path.argtypes = pre_args + [ci]
+        lib.mhc_pre_with_path.restype = ci
+        lib.mhc_pre_path_for.argtypes = [i64, ci, ci, ci]
+        lib.mhc_pre_path_for.restype = ci
+        lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
+        lib.mhc_post.restype = ci
+        lib.mhc_status_string.argtypes = [ci]
+        lib.mhc_status_string.restype = ctypes.c_char_p
+        lib.mhc_last_error.argtypes = []
+        lib.mhc_last_error.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        lib = load_library()
+        detail = lib.mhc_status_string(status).decode()
+        if status == 6:
+            detail += "; " + lib.mhc_last_error().decode()
+        raise MhcError(status, where, detail)
+
+
+def _dt(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return MHC_BF16
+    if t.dtype == torch.float32:
+        return MHC_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t, name, dtype=None, device=None) -> int:
+    import torch
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch tensor or raw device pointer")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (the library takes device pointers)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream, device) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def mhc_pre_with_path(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+                      eps, t_max, x_in, H, stream=None, path: int = PRE_AUTO):
+    """Pre stage on an explicit kernel path (see mhc_pre)."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    f32 = torch.float32
+    ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
+                b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
+                b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
+                H=_ptr(H, "H", f32, dev))
+    m = n * n + 2 * n
+    if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m):
+        raise ValueError("mhc_pre: shapes must be phi [n*d, m], x_in [T, d], H [T, m]")
+    if b_pre.numel() != n or b_post.numel() != n or b_res.numel() != n * n:
+        raise ValueError("mhc_pre: b_pre/b_post need n entries, b_res n*n")
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_pre_with_path(ptrs["X"], ptrs["phi"], ptrs["b_pre"], ptrs["b_post"],
+                                   ptrs["b_res"], float(alpha_pre), float(alpha_post),
+                                   float(alpha_res), T, n, d, float(eps), int(t_max), _dt(X),
+                                   ptrs["x_in"], ptrs["H"], _stream(stream, dev), int(path))
+    _check(st, "mhc_pre")
+
+
+def mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
+            x_in, H, stream=None):
+    """Pre stage: x_in = H_pre X and H = [H_pre | H_res | H_post] for every token.
+
+    X [T, n, d] (bf16/fp32), phi [n*d, n*n+2n] fp32, b_pre/b_post [n], b_res [n, n] fp32;
+    outputs x_in [T, d] (X's dtype) and H [T, n*n+2n] fp32, written in place."""
+    mhc_pre_with_path(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps,
+                      t_max, x_in, H, stream, PRE_AUTO)
+
+
+def mhc_post(X, F_out, H, X_out, stream=None):
+    """Post stage: X_out = H_res X + H_post^T F_out for every token (written in place)."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    px = _ptr(X, "X", device=dev)
+    pf = _ptr(F_out, "F_out", X.dtype, dev)
+    ph = _ptr(H, "H", torch.float32, dev)
+    po = _ptr(X_out, "X_out", X.dtype, dev)
+    if tuple(F_out.shape) != (T, d) or tuple(H.shape) != (T, n * n + 2 * n) or \
+            tuple(X_out.shape) != (T, n, d):
+        raise ValueError("mhc_post: shapes must be F_out [T, d], H [T, m], X_out [T, n, d]")
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_post(px, pf, ph, T, n, d, _dt(X), po, _stream(stream, dev))
+    _check(st, "mhc_post")
+
+
+def mhc_pre_path_for(T: int, n: int, d: int, dtype) -> int:
+    """Kernel path mhc_pre would take on the current device (PRE_GENERIC / PRE_CLUSTER_TC)."""
+    import torch
+    dt = dtype if isinstance(dtype, int) else (MHC_BF16 if dtype == torch.bfloat16 else MHC_F32)
+    return int(load_library().mhc_pre_path_for(int(T), int(n), int(d), dt))

@@ -1,0 +1,58 @@
+// launch.cuh -- internal launcher interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mhc {
+
+enum DType { F32 = 0, BF16 = 1 };
+
+struct PreArgs {
+    const void* X;
+    const float* phi;
+    const float* b_pre;
+    const float* b_post;
+    const float* b_res;
+    float a_pre, a_post, a_res;
+    int64_t T;
+    int n, d;
+    float eps;
+    int t_max;
+    DType dt;
+    void* x_in;
+    float* H;
+    cudaStream_t stream;
+};
+
+struct PostArgs {
+    const void* X;
+    const void* F;
+    const float* H;
+    int64_t T;
+    int n, d;
+    DType dt;
+    void* Y;
+    cudaStream_t stream;
+};
+
+// Per-device launch limits, queried once per device and cached.
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int max_smem_optin;
+    int cc_major, cc_minor;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+cudaError_t launch_pre_generic(const PreArgs& a);
+
+// Cluster tensor-core path: shape test (host only) and launch.
+bool pre_cluster_tc_shape_ok(int64_t T, int n, int d, DType dt);
+// Whether the current device can run it (sm_100 and a resident 16-CTA cluster).
+bool pre_cluster_tc_device_ok();
+cudaError_t launch_pre_cluster_tc(const PreArgs& a);
+
+cudaError_t launch_post(const PostArgs& a);
+
+}  // namespace mhc

@@ -1,0 +1,143 @@
+// pre_generic.cu -- CUDA-core kernel for the mHC pre stage: any n <= 8, any d, f32 or bf16.
+//
+// Per CTA a tile of TT tokens:
+//   1. K loop (K = n*d): stage X[tile, k0:k0+KC] (as fp32) and phi[k0:k0+KC, :] in shared
+//      memory; accumulate the projection h = v . phi (fp32) and the sum of squares of v.
+//   2. One thread per token turns h into [H_pre | H_res | H_post] ("DeepSeek-V4/mhc",
+//      equations rmsnorm, a/b/c-tilde, gate, sinkhorn) and writes H.
+//   3. x_in = sum_i H_pre[i] X[t, i, :] (slavadubrov.com Eq. 3, read map on raw X).
+// Exact fp32 arithmetic with fp32 phi: this is the path for fp32 storage and for shapes
+// the tensor-core path does not take.
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace mhc {
+namespace {
+
+constexpr int TT = 16;        // tokens per CTA
+constexpr int KC = 64;        // K chunk staged per step
+constexpr int THREADS = 256;
+
+template <int N, typename T>
+__global__ void __launch_bounds__(THREADS)
+pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
+                   const float* __restrict__ b_pre, const float* __restrict__ b_post,
+                   const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
+                   int64_t Tn, int d, float eps, int t_max, T* __restrict__ x_in,
+                   float* __restrict__ H)
+{
+    constexpr int M = N * N + 2 * N;
+    constexpr int NO = (TT * M + THREADS - 1) / THREADS;   // projection outputs per thread
+    __shared__ float xs[TT][KC + 1];
+    __shared__ float ps[KC][M];
+    __shared__ float hs[TT][M];
+    __shared__ float ss_s[TT];
+    __shared__ float hpre_s[TT][N];
+
+    const int K = N * d;
+    const int64_t t0 = (int64_t)blockIdx.x * TT;
+    const int tid = threadIdx.x;
+
+    float acc[NO];
+#pragma unroll
+    for (int r = 0; r < NO; ++r) acc[r] = 0.f;
+    float ssq = 0.f;                                  // partial sum of squares, token tid/16
+    const int my_t = tid / (THREADS / TT);            // 16 threads per token when staging
+    const int my_k0 = (tid % (THREADS / TT)) * (KC * TT / THREADS);
+    const int64_t my_tok = t0 + my_t;
+
+    for (int k0 = 0; k0 < K; k0 += KC) {
+#pragma unroll
+        for (int u = 0; u < KC * TT / THREADS; ++u) {
+            const int kk = my_k0 + u;
+            const int k = k0 + kk;
+            float v = 0.f;
+            if (my_tok < Tn && k < K) v = to_f32(X[my_tok * K + k]);
+            xs[my_t][kk] = v;
+            ssq = fmaf(v, v, ssq);
+        }
+        for (int e = tid; e < KC * M; e += THREADS) {
+            const int kk = e / M, j = e - kk * M;
+            const int k = k0 + kk;
+            ps[kk][j] = (k < K) ? phi[(int64_t)k * M + j] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < NO; ++r) {
+            const int o = tid + THREADS * r;
+            if (o < TT * M) {
+                const int t = o / M, j = o - t * M;
+                float a = acc[r];
+#pragma unroll 8
+                for (int kk = 0; kk < KC; ++kk) a = fmaf(xs[t][kk], ps[kk][j], a);
+                acc[r] = a;
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < NO; ++r) {
+        const int o = tid + THREADS * r;
+        if (o < TT * M) hs[o / M][o % M] = acc[r];
+    }
+    // sum of squares: the 16 threads of a token are one half-warp
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+    if ((tid & 15) == 0) ss_s[my_t] = ssq;
+    __syncthreads();
+
+    if (tid < TT && t0 + tid < Tn) {
+        const int64_t tok = t0 + tid;
+        const float r = sqrtf(ss_s[tid] / (float)K + eps);
+        float out[M];
+        token_maps<N>(hs[tid], 1.0f / r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+#pragma unroll
+        for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
+#pragma unroll
+        for (int i = 0; i < N; ++i) hpre_s[tid][i] = out[i];
+    }
+    __syncthreads();
+
+    for (int e = tid; e < TT * d; e += THREADS) {
+        const int t = e / d, c = e - t * d;
+        const int64_t tok = t0 + t;
+        if (tok >= Tn) break;
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) a = fmaf(hpre_s[t][i], to_f32(X[tok * K + (int64_t)i * d + c]), a);
+        store_elem(&x_in[tok * d + c], a);
+    }
+}
+
+template <int N, typename T>
+cudaError_t launch_n(const PreArgs& a) {
+    const int64_t blocks = (a.T + TT - 1) / TT;
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    pre_generic_kernel<N, T><<<(unsigned)blocks, THREADS, 0, a.stream>>>(
+        static_cast<const T*>(a.X), a.phi, a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post,
+        a.a_res, a.T, a.d, a.eps, a.t_max, static_cast<T*>(a.x_in), a.H);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const PreArgs& a) {
+    switch (a.n) {
+        case 1: return launch_n<1, T>(a);
+        case 2: return launch_n<2, T>(a);
+        case 3: return launch_n<3, T>(a);
+        case 4: return launch_n<4, T>(a);
+        case 5: return launch_n<5, T>(a);
+        case 6: return launch_n<6, T>(a);
+        case 7: return launch_n<7, T>(a);
+        case 8: return launch_n<8, T>(a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pre_generic(const PreArgs& a) {
+    return a.dt == BF16 ? launch_t<__nv_bfloat16>(a) : launch_t<float>(a);
+}
+
+}  // namespace mhc

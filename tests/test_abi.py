@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every symbol include/mhc.h declares, and rejects bad
+arguments on the host (status codes, no launch).  No compute call runs here: every call
+below fails validation before the library touches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mhc_hyper_connections_b200 as mhc
+from mhc_hyper_connections_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return mhc.load_library()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "mhc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(mhc_\w+)\s*\(", src))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert declared == set(mhc.EXPORTED_SYMBOLS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.mhc_status_string(code)
+        assert s and s.decode() != "unknown status"
+    assert lib.mhc_status_string(99).decode() == "unknown status"
+    assert lib.mhc_last_error().decode() == ""
+
+
+# fake, never-dereferenced addresses: validation rejects before any CUDA call
+A = 0x10000000
+
+
+def _pre(lib, X=A, phi=A + 0x1000000, bp=A + 0x2000000, bq=A + 0x2000100, br=A + 0x2000200,
+         T=4, n=4, d=64, t_max=20, dt=1, x_in=A + 0x3000000, H=A + 0x4000000):
+    return lib.mhc_pre(X, phi, bp, bq, br, 0.01, 0.01, 0.01, T, n, d, 1e-20, t_max, dt, x_in, H, None)
+
+
+def test_pre_validation(lib):
+    assert _pre(lib, T=0) == 0                       # T = 0 is a no-op
+    assert _pre(lib, T=0, X=0, x_in=0, H=0) == 0     # ... even with NULL buffers
+    assert _pre(lib, n=0) == 2 and _pre(lib, n=9) == 2
+    assert _pre(lib, d=0) == 2 and _pre(lib, T=-1) == 2
+    assert _pre(lib, t_max=-1) == 2 and _pre(lib, t_max=1001) == 2
+    assert _pre(lib, dt=2) == 4
+    assert _pre(lib, X=0) == 1 and _pre(lib, H=0) == 1 and _pre(lib, phi=0) == 1
+    assert _pre(lib, br=0) == 1
+    assert _pre(lib, X=A + 1) == 3                   # bf16 needs 2-byte alignment
+    assert _pre(lib, dt=0, X=A + 2) == 3             # fp32 needs 4
+    assert _pre(lib, H=A + 0x4000002) == 3
+    assert _pre(lib, x_in=A + 16) == 7               # x_in overlaps X
+    assert _pre(lib, H=A + 0x3000010) == 7           # H overlaps x_in
+    assert _pre(lib, H=A + 0x1000000) == 7           # H overlaps phi
+    huge = (1 << 62) // (4 * 64)
+    assert _pre(lib, T=huge) == 2                    # byte counts would overflow
+
+
+def test_pre_with_path_rejects_unknown_path(lib):
+    st = lib.mhc_pre_with_path(A, A + 0x1000000, A + 0x2000000, A + 0x2000100, A + 0x2000200,
+                               0.01, 0.01, 0.01, 4, 4, 64, 1e-20, 20, 1, A + 0x3000000,
+                               A + 0x4000000, None, 7)
+    assert st == 5
+
+
+def test_post_validation(lib):
+    def post(X=A, F=A + 0x1000000, H=A + 0x2000000, T=4, n=4, d=64, dt=1, Y=A + 0x3000000):
+        return lib.mhc_post(X, F, H, T, n, d, dt, Y, None)
+    assert post(T=0) == 0
+    assert post(n=0) == 2 and post(d=-3) == 2
+    assert post(dt=7) == 4
+    assert post(Y=0) == 1 and post(F=0) == 1
+    assert post(X=A + 1) == 3
+    assert post(Y=A + 64) == 7                       # X_out overlaps X
+    assert post(Y=A + 0x1000000) == 7                # X_out overlaps F_out
+
+
+def test_binding_refuses_host_tensors():
+    torch = pytest.importorskip("torch")
+    X = torch.zeros(2, 4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mhc.mhc_post(X, torch.zeros(2, 8, dtype=torch.bfloat16), torch.zeros(2, 24),
+                     torch.zeros_like(X))
+
+
+def test_path_query_on_cpu_host(lib):
+    # With no usable GPU the query answers the generic path and launches nothing.
+    assert lib.mhc_pre_path_for(16, 4, 64, 0) == mhc.PRE_GENERIC
