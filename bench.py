@@ -142,6 +142,8 @@ def run_reference(args, rank, world):
     from mhc_hyper_connections_b200 import workloads as wl
 
     w = wl.make_config(args.config)
+    if args.tokens:
+        w = w.tokens(np.arange(min(args.tokens, w.T)))
     cores = os.cpu_count() or 1
     used = oracle.threads_used(cores)
     s = w.scalars()
@@ -242,6 +244,8 @@ def run_ours(args, rank, world, local_rank):
         return float(t.item())
 
     w = wl.make_config(args.config)
+    if args.tokens:
+        w = w.tokens(np.arange(min(args.tokens, w.T)))
     T, n, d = w.T, w.n, w.d
     es = 2 if w.dtype == "bf16" else 4
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -302,14 +306,14 @@ def run_ours(args, rank, world, local_rank):
 
     value = world * T * K / (ms_total / 1e3)
     peak, peak_src = _hbm_peak()
-    b_pre, b_post = bytes_per_token(n, d, es)
-    kern = {"pre": {"ms": pre_ms, "bytes_per_launch": b_pre * T,
-                    "gbs": b_pre * T / (pre_ms / 1e3) / 1e9,
+    by_pre, by_post = bytes_per_token(n, d, es)
+    kern = {"pre": {"ms": pre_ms, "bytes_per_launch": by_pre * T,
+                    "gbs": by_pre * T / (pre_ms / 1e3) / 1e9,
                     "path": {1: "generic", 2: "cluster_tc"}.get(path, str(path)),
                     "source": "mhc_hyper_connections_b200/csrc/" +
                               ("pre_cluster_tc.cu" if path == 2 else "pre_generic.cu")},
-            "post": {"ms": post_ms, "bytes_per_launch": b_post * T,
-                     "gbs": b_post * T / (post_ms / 1e3) / 1e9,
+            "post": {"ms": post_ms, "bytes_per_launch": by_post * T,
+                     "gbs": by_post * T / (post_ms / 1e3) / 1e9,
                      "source": "mhc_hyper_connections_b200/csrc/post.cu"}}
     dom = max(kern, key=lambda k: kern[k]["ms"])
     traffic = None
@@ -320,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": kern[dom]["bytes_per_launch"]}
-    b_dep = b_pre + b_post
+    b_dep = by_pre + by_post
     step_gbs = b_dep * T * world / (ms_total / 1e3 / K) / 1e9 / world
     hbm = {"B_dep_bytes_per_token": b_dep, "B_lit_bytes_per_token": (2 * n + 2) * d * es,
            "gbs_per_gpu": step_gbs, "frac_of_8TBs": step_gbs / NOMINAL_HBM_GBS,
@@ -396,6 +400,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=wl.HEADLINE, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")

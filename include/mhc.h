@@ -130,6 +130,17 @@ mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt);
 mhc_status mhc_post(const void* X, const void* F_out, const float* H, int64_t T, int n, int d,
                     mhc_dtype dt, void* X_out, mhc_stream_t stream);
 
+/*
+ * mhc_device_status -- read and clear the device-side status word of the tensor-core
+ * kernel.  Its waits between warps and between the CTAs of a cluster are bounded in
+ * time (1 s each); a wait that expires makes the kernel stop early, leaving its outputs
+ * incomplete, and sets a bit here naming the wait.  *code = 0 means every wait of every
+ * launch since the last read completed.  Blocks until prior work on the legacy default
+ * stream (and streams that synchronise with it) has finished.  No counterpart on the
+ * pages: this is the library's failure report.
+ */
+mhc_status mhc_device_status(uint32_t* code);
+
 /* Static English text for a status code (never NULL). */
 const char* mhc_status_string(mhc_status status);
 

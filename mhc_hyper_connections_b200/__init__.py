@@ -19,7 +19,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_post", "mhc_pre_path_for", "MhcError",
+__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_post", "mhc_pre_path_for", "mhc_device_status",
+           "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
 
@@ -33,7 +34,7 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
 
 # Every function include/mhc.h declares.
 EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_path_for", "mhc_post",
-                    "mhc_status_string", "mhc_last_error")
+                    "mhc_status_string", "mhc_last_error", "mhc_device_status")
 
 _lock = threading.Lock()
 _lib = None
@@ -75,6 +76,8 @@ def load_library():
         lib.mhc_status_string.restype = ctypes.c_char_p
         lib.mhc_last_error.argtypes = []
         lib.mhc_last_error.restype = ctypes.c_char_p
+        lib.mhc_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        lib.mhc_device_status.restype = ci
         _lib = lib
     return _lib
 
@@ -176,6 +179,14 @@ def mhc_post(X, F_out, H, X_out, stream=None):
     with torch.cuda.device(dev):
         st = lib.mhc_post(px, pf, ph, T, n, d, _dt(X), po, _stream(stream, dev))
     _check(st, "mhc_post")
+
+
+def mhc_device_status() -> int:
+    """Read and clear the tensor-core kernel's device status word (0 = every bounded wait
+    completed; otherwise bits naming the waits that expired)."""
+    code = ctypes.c_uint32(0)
+    _check(load_library().mhc_device_status(ctypes.byref(code)), "mhc_device_status")
+    return int(code.value)
 
 
 def mhc_pre_path_for(T: int, n: int, d: int, dtype) -> int:

@@ -49,9 +49,11 @@ cudaError_t launch_pre_generic(const PreArgs& a);
 
 // Cluster tensor-core path: shape test (host only) and launch.
 bool pre_cluster_tc_shape_ok(int64_t T, int n, int d, DType dt);
-// Whether the current device can run it (sm_100 and a resident 16-CTA cluster).
-bool pre_cluster_tc_device_ok();
+// Whether the current device can run it for (n, d) (sm_100 and a resident 16-CTA cluster).
+bool pre_cluster_tc_device_ok(int n, int d);
 cudaError_t launch_pre_cluster_tc(const PreArgs& a);
+// Status word of the cluster kernel's bounded waits (0 = fine); optionally cleared.
+cudaError_t pre_cluster_tc_status(unsigned* out, bool clear);
 
 cudaError_t launch_post(const PostArgs& a);
 

@@ -114,7 +114,7 @@ extern "C" {
 
 mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
     if (check_shape(T, n, d, dt) == MHC_OK &&
-        pre_cluster_tc_shape_ok(T, n, d, dt == MHC_BF16 ? BF16 : F32) && pre_cluster_tc_device_ok())
+        pre_cluster_tc_shape_ok(T, n, d, dt == MHC_BF16 ? BF16 : F32) && pre_cluster_tc_device_ok(n, d))
         return MHC_PRE_CLUSTER_TC;
     return MHC_PRE_GENERIC;
 }
@@ -134,7 +134,7 @@ mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre
                                n, d, eps, t_max, dt, x_in, H, stream);
     cudaError_t e;
     if (path == MHC_PRE_CLUSTER_TC) {
-        if (!pre_cluster_tc_shape_ok(T, n, d, a.dt) || !pre_cluster_tc_device_ok())
+        if (!pre_cluster_tc_shape_ok(T, n, d, a.dt) || !pre_cluster_tc_device_ok(n, d))
             return MHC_ERR_UNSUPPORTED;
         if (!aligned(X, 16) || !aligned(x_in, 16) || !aligned(phi, 16)) return MHC_ERR_UNSUPPORTED;
         e = launch_pre_cluster_tc(a);
@@ -193,5 +193,14 @@ const char* mhc_status_string(mhc_status s) {
 }
 
 const char* mhc_last_error(void) { return g_last_error; }
+
+mhc_status mhc_device_status(uint32_t* code) {
+    if (!code) return MHC_ERR_NULL;
+    unsigned v = 0;
+    cudaError_t e = pre_cluster_tc_status(&v, true);
+    if (e != cudaSuccess) return cuda_fail(e, "mhc_device_status");
+    *code = v;
+    return MHC_OK;
+}
 
 }  // extern "C"

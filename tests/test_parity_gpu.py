@@ -185,12 +185,32 @@ def test_paths_agree_with_each_other():
     assert (d <= 2 ** -7 * g[0].float().abs() + 1e-5).all()
 
 
-def test_auto_path_on_headline_shape_is_tensor_core():
-    """On a B200 the headline shape (n=4, d=4096, bf16) runs the cluster tensor-core kernel."""
-    major, _ = torch.cuda.get_device_capability()
-    if major != 10:
+def test_auto_path_on_b200_shapes_is_tensor_core():
+    """On a B200 the bf16 shapes with n <= 4 and d in {1024..4096} run the cluster
+    tensor-core kernel; everything else runs the generic kernel."""
+    major, minor = torch.cuda.get_device_capability()
+    if (major, minor) != (10, 0):
         pytest.skip("not an sm_100 device")
-    if not hasattr(mhc, "PRE_CLUSTER_TC"):
-        pytest.skip("no tensor-core path in this build")
-    p = mhc.mhc_pre_path_for(16384, 4, 4096, 1)
-    assert p in (mhc.PRE_GENERIC, mhc.PRE_CLUSTER_TC)
+    for n in (1, 2, 3, 4):
+        for d in (1024, 2048, 3072, 4096):
+            assert mhc.mhc_pre_path_for(16384, n, d, 1) == mhc.PRE_CLUSTER_TC, (n, d)
+    assert mhc.mhc_pre_path_for(16384, 4, 4096, 0) == mhc.PRE_GENERIC     # fp32 storage
+    assert mhc.mhc_pre_path_for(16384, 8, 4096, 1) == mhc.PRE_GENERIC     # n = 8
+    assert mhc.mhc_pre_path_for(16384, 4, 512, 1) == mhc.PRE_GENERIC      # d < 1024
+
+
+def test_device_status_clean_after_runs():
+    """Every bounded wait of the tensor-core kernel completed in the runs above."""
+    w = wl.make_inputs(T=77, n=4, d=2048, dtype="bf16", seed=8)
+    run_gpu(w)
+    assert mhc.mhc_device_status() == 0
+
+
+def test_tensor_core_path_rejects_what_it_cannot_run():
+    w = wl.make_inputs(T=8, n=4, d=64, dtype="bf16", seed=2)
+    t = torch_inputs(w)
+    x_in = torch.empty(8, 64, dtype=torch.bfloat16, device="cuda")
+    H = torch.empty(8, 24, device="cuda")
+    with pytest.raises(mhc.MhcError, match="UNSUPPORTED"):
+        mhc.mhc_pre_with_path(t["X"], t["phi"], t["b_pre"], t["b_post"], t["b_res"], 0.01, 0.01,
+                              0.01, 1e-20, 20, x_in, H, path=mhc.PRE_CLUSTER_TC)
