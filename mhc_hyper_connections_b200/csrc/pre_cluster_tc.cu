@@ -25,6 +25,10 @@
 //
 // Warp roles (512 threads): 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2 owner
 // reduction, 3 Sinkhorn / H writer, 4-7 TMEM epilogue, 8-11 sum of squares, 12-15 x_in.
+// Issuing a tcgen05.mma costs the issuing thread ~100 cycles whatever the shape, so four
+// warps issue a tile's MMAs, each into its own TMEM accumulator; the epilogue adds the
+// accumulators in a fixed order and ships each owner its rows with one bulk
+// shared-to-shared copy.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records the failing
 // wait in a status word, drains its own copies in flight, frees TMEM and returns.
 #include <cuda.h>
@@ -46,7 +50,11 @@ namespace tc {
 constexpr int S = 16;          // CTAs per cluster
 constexpr int NT = 16;         // tokens per tile (MMA N)
 constexpr int MAXST = 8;       // max shared-memory stages
-constexpr int THREADS = 512;
+constexpr int NMMA = 4;        // warps issuing tcgen05.mma (issue cost is per thread)
+constexpr int THREADS = 512 + 32 * (NMMA - 1);
+constexpr int NSLOT = 4;       // depth of the cross-CTA rings (partials in, H_pre out)
+constexpr int NACC = 2;        // TMEM accumulator buffers (tile k uses buffer k % NACC)
+constexpr int MAXCHAIN = NMMA; // one accumulation chain per MMA warp
 constexpr int RING = 64;       // logits ring (2 batches of 32 tokens)
 constexpr int BATCH = 32;
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait, then give up
@@ -71,9 +79,9 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >
 // barrier slots (8 bytes each) inside the barrier block
 enum : int {
     B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = 3 * MAXST,
-    B_PART_FULL = 4 * MAXST, B_PART_EMPTY = B_PART_FULL + 2, B_HPRE_FULL = B_PART_EMPTY + 2,
-    B_HPRE_EMPTY = B_HPRE_FULL + 2, B_LG_FULL = B_HPRE_EMPTY + 2, B_LG_EMPTY = B_LG_FULL + 2,
-    B_COUNT = B_LG_EMPTY + 2
+    B_PART_FULL = 4 * MAXST, B_PART_EMPTY = B_PART_FULL + NSLOT,
+    B_HPRE_FULL = B_PART_EMPTY + NSLOT, B_HPRE_EMPTY = B_HPRE_FULL + NSLOT,
+    B_LG_FULL = B_HPRE_EMPTY + NSLOT, B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
 };
 
 // status codes: which wait expired
@@ -108,11 +116,24 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
 }
-// arrive on an mbarrier of another CTA of the cluster (shared::cluster address)
+// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).  Used
+// only to say "this buffer may be overwritten": every value read from the buffer has
+// been consumed by an instruction before the arrive, so no release fence is needed (a
+// release here would also wait for this warp's earlier global stores).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cbar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cbar) : "memory");
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(cbar) : "memory");
 }
+// CTA-scope acquire: barriers completed by this CTA's own threads, TMA or tensor cores
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// cluster-scope acquire: barriers whose phase completes with data st.async'd by peers
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
                  "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
@@ -134,6 +155,18 @@ __device__ __forceinline__ void st_async_f32(uint32_t raddr, float a, uint32_t r
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
                  :: "r"(raddr), "f"(a), "r"(rbar) : "memory");
 }
+// bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into a peer's,
+// completing `bytes` of transaction count on the peer's mbarrier
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                             uint32_t rbar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(rbar) : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_allbut1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2) {
     asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -193,12 +226,14 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 
 // Bounded wait: true when the phase completed; false when the CTA is aborting or the
 // wait expired (then the status word and the CTA's abort flag are set).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            unsigned code, bool honour_abort = true) {
-    if (mbar_try(bar, parity)) return true;
+    auto try_once = [&]() { return CLUSTER ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity); };
+    if (try_once()) return true;
     const uint64_t t0 = gtimer();
     while (true) {
-        if (mbar_try(bar, parity)) return true;
+        if (try_once()) return true;
         if (honour_abort && *abort_flag) return false;
         if (gtimer() - t0 > kWaitNs) {
             atomicOr(&g_pre_tc_status, code);
@@ -215,7 +250,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                       const float* __restrict__ b_pre, const float* __restrict__ b_post,
                       const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                       int T, int d, float eps, int t_max, __nv_bfloat16* __restrict__ x_in,
-                      float* __restrict__ H, int ncb, int nstage, int tmem_cols)
+                      float* __restrict__ H, int ncb, int nstage, int nchain, int tmem_cols)
 {
     using C = Cfg<N>;
     constexpr int M = C::M;
@@ -234,9 +269,10 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     uint32_t off = 0;
     const uint32_t o_phi = off;  off += (uint32_t)KA * C::ATOM_PHI;
     const uint32_t o_x = off;    off += (uint32_t)nstage * stage_bytes;
-    const uint32_t o_recv = off; off += 2u * S * C::RECV_STRIDE * 4u;
-    const uint32_t o_hpre = off; off += 2u * NT * 16u;
+    const uint32_t o_recv = off; off += (uint32_t)NSLOT * S * C::RECV_STRIDE * 4u;
+    const uint32_t o_hpre = off; off += (uint32_t)NSLOT * NT * 16u;
     const uint32_t o_ring = off; off += (uint32_t)RING * M * 4u;
+    const uint32_t o_stg = off;  off += 4u * 2u * NT * 16u * 4u;     // epilogue staging, per warp x2
     off = (off + 15u) & ~15u;
     const uint32_t o_bar = off;  off += B_COUNT * 8u;
     const uint32_t o_misc = off;
@@ -255,17 +291,21 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
             mbar_init(bar(B_FULL + s), 1);
-            mbar_init(bar(B_EMPTY + s), 9);       // MMA commit + 4 sum-of-squares + 4 x_in warps
-            mbar_init(bar(B_ACCF + s), 1);
-            mbar_init(bar(B_ACCE + s), 4);        // 4 epilogue warps
+            mbar_init(bar(B_EMPTY + s), NMMA + 8);   // MMA warps + 4 sum-of-squares + 4 x_in
         }
-        for (int sl = 0; sl < 2; ++sl) {
+        for (int ab = 0; ab < NACC; ++ab) {
+            mbar_init(bar(B_ACCF + ab), NMMA);
+            mbar_init(bar(B_ACCE + ab), 4);       // 4 epilogue warps
+        }
+        for (int sl = 0; sl < NSLOT; ++sl) {
             mbar_init(bar(B_PART_FULL + sl), 1);
             mbar_init(bar(B_PART_EMPTY + sl), S);        // one arrive per owner CTA
             mbar_init(bar(B_HPRE_FULL + sl), 1);
             mbar_init(bar(B_HPRE_EMPTY + sl), S * 4);    // 4 x_in warps of every CTA
-            mbar_init(bar(B_LG_FULL + sl), 1);
-            mbar_init(bar(B_LG_EMPTY + sl), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_LG_FULL + b), 1);
+            mbar_init(bar(B_LG_EMPTY + b), 1);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -294,7 +334,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int sl = 0; sl < 2; ++sl) {
+        for (int sl = 0; sl < NSLOT; ++sl) {
             mbar_arrive_tx(bar(B_PART_FULL + sl), C::TX_PART);
             mbar_arrive_tx(bar(B_HPRE_FULL + sl), C::TX_HPRE);
         }
@@ -328,31 +368,32 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                 wait_phase(bar(B_FULL + k % nstage), (k / nstage) & 1, abort_flag, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // MMA issuer
+    } else if (warp == 1 || warp >= 16) {
+        // MMA issuers: warp mw issues the K atoms a = mw, mw + nchain, ... into chain mw
+        const int mw = warp == 1 ? 0 : warp - 15;
         if (lane == 0) {
             int issued = 0;
             for (int k = 0; k < my_tiles; ++k) {
-                const int s = k % nstage, u = k / nstage;
+                const int s = k % nstage, u = k / nstage, ab = k % NACC, ua = k / NACC;
                 if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_MMA)) break;
-                if (!wait_phase(bar(B_ACCE + s), (u & 1) ^ 1, abort_flag, E_ACCE)) break;
+                if (!wait_phase(bar(B_ACCE + ab), (ua & 1) ^ 1, abort_flag, E_ACCE)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(s * NT);
+                const uint32_t d_tmem = tmem + (uint32_t)(ab * nchain * NT);
                 const uint32_t xs = base + o_x + (uint32_t)s * stage_bytes;
-                for (int a = 0; a < KA; ++a) {
+                for (int a = mw; a < KA && mw < nchain; a += nchain) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = sw128_desc(base + o_phi + (uint32_t)a * C::ATOM_PHI + kk * 32);
                         const uint64_t bd = sw128_desc(xs + (uint32_t)a * (NT * 128) + kk * 32);
-                        mma_bf16(d_tmem, ad, bd, (a | kk) != 0);
+                        mma_bf16(d_tmem + (uint32_t)(mw * NT), ad, bd, (a != mw) || kk);
                     }
                 }
                 mma_commit(bar(B_EMPTY + s));
-                mma_commit(bar(B_ACCF + s));
+                mma_commit(bar(B_ACCF + ab));
                 issued = k + 1;
             }
             if (issued > 0)   // all MMAs complete before TMEM is released
-                wait_phase(bar(B_ACCF + (issued - 1) % nstage), ((issued - 1) / nstage) & 1,
+                wait_phase(bar(B_ACCF + (issued - 1) % NACC), ((issued - 1) / NACC) & 1,
                            abort_flag, E_DRAIN, false);
         }
         __syncwarp();
@@ -360,8 +401,8 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
         // owner: reduce the 16 partials of this CTA's token, broadcast H_pre, queue logits
         const float invK = 1.0f / (float)(N * d);
         for (int k = 0; k < my_tiles; ++k) {
-            const int sl = k & 1, v = k >> 1;
-            if (!wait_phase(bar(B_PART_FULL + sl), v & 1, abort_flag, E_PART_FULL)) break;
+            const int sl = k % NSLOT, v = k / NSLOT;
+            if (!wait_phase<true>(bar(B_PART_FULL + sl), v & 1, abort_flag, E_PART_FULL)) break;
             const float* rb = recv + sl * S * C::RECV_STRIDE;
             float ss = 0.f;
 #pragma unroll
@@ -439,38 +480,54 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             if (lane == 0) mbar_arrive(bar(B_LG_EMPTY + b));
         }
     } else if (warp < 8) {
-        // TMEM epilogue: partial projections -> owners (st.async into their receive slot)
+        // TMEM epilogue: sum the accumulation chains, stage this warp's 16 rows of the
+        // tile's partial projections, and bulk-copy token t's rows to owner CTA t
         const int q = warp & 3;
+        const bool has_rows = 16 * q < C::RECV_D;
+        const uint32_t nbytes = (uint32_t)min(16, C::RECV_D - 16 * q) * 4u;
+        float* stg = reinterpret_cast<float*>(sb + o_stg) + q * (2 * NT * 16);
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         for (int k = 0; k < my_tiles; ++k) {
-            const int s = k % nstage, u = k / nstage, sl = k & 1, v = k >> 1;
-            if (!wait_phase(bar(B_ACCF + s), u & 1, abort_flag, E_ACCF)) break;
+            const int ab = k % NACC, ua = k / NACC, sl = k % NSLOT, v = k / NSLOT;
+            if (!wait_phase(bar(B_ACCF + ab), ua & 1, abort_flag, E_ACCF)) break;
             tc_fence_after();
             float dv[16];
-            if (16 * q < C::RECV_D) tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(s * NT), dv);
+            if (has_rows) {
+                tmem_ld16(tq + (uint32_t)(ab * nchain * NT), dv);
+                for (int c = 1; c < nchain; ++c) {
+                    float e[16];
+                    tmem_ld16(tq + (uint32_t)((ab * nchain + c) * NT), e);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) dv[t] += e[t];
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_ACCE + s));
-            if (16 * q >= C::RECV_D) continue;
-            if (!wait_phase(bar(B_PART_EMPTY + sl), (v & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
-            const int p = lane & 3;
-            const bool sender = lane < 4 && (16 * q + 4 * p) < C::RECV_D;
-            const uint32_t slot_off = (uint32_t)((sl * S + (int)rank) * C::RECV_STRIDE + 16 * q + 4 * p) * 4u;
+            if (lane == 0) mbar_arrive(bar(B_ACCE + ab));
+            if (!has_rows) continue;
+            float* sbuf = stg + (k & 1) * (NT * 16);
+            if (lane < NT) bulk_wait_read_allbut1();     // copies out of sbuf two tiles ago done
+            __syncwarp();
+            if (lane < 16) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float g0 = __shfl_sync(0xffffffffu, dv[t], 4 * p + 0);
-                const float g1 = __shfl_sync(0xffffffffu, dv[t], 4 * p + 1);
-                const float g2 = __shfl_sync(0xffffffffu, dv[t], 4 * p + 2);
-                const float g3 = __shfl_sync(0xffffffffu, dv[t], 4 * p + 3);
-                if (sender)
-                    st_async_v4(mapa(base + o_recv + slot_off, t), g0, g1, g2, g3,
-                                mapa(bar(B_PART_FULL + sl), t));
+                for (int t = 0; t < NT; ++t) sbuf[t * 16 + lane] = dv[t];
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (!wait_phase(bar(B_PART_EMPTY + sl), (v & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
+            if (lane < NT) {
+                const uint32_t dst = base + o_recv +
+                                     (uint32_t)((sl * S + (int)rank) * C::RECV_STRIDE + 16 * q) * 4u;
+                bulk_to_peer(mapa(dst, lane), smem_u32(sbuf + lane * 16), nbytes,
+                             mapa(bar(B_PART_FULL + sl), lane));
             }
         }
+        if (lane < NT) bulk_wait_all();
     } else if (warp < 12) {
         // sum of squares of this CTA's slice of every token of the tile -> owners
         const int t = (warp - 8) * 4 + (lane >> 3), u8 = lane & 7;
         for (int k = 0; k < my_tiles; ++k) {
-            const int s = k % nstage, u = k / nstage, sl = k & 1, v = k >> 1;
+            const int s = k % nstage, u = k / nstage, sl = k % NSLOT, v = k / NSLOT;
             if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_SS)) break;
             const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
             float ss = 0.f;
@@ -498,10 +555,10 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
         const int t = (warp - 12) * 4 + (lane >> 3), u8 = lane & 7;
         const int coff = (int)rank * cpc + (u8 << 3);
         for (int k = 0; k < my_tiles; ++k) {
-            const int s = k % nstage, u = k / nstage, sl = k & 1, v = k >> 1;
+            const int s = k % nstage, u = k / nstage, sl = k % NSLOT, v = k / NSLOT;
             const int64_t tok = (int64_t)(cid + k * ncl) * NT + t;
             if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_XIN)) break;
-            if (!wait_phase(bar(B_HPRE_FULL + sl), v & 1, abort_flag, E_HPRE_FULL)) break;
+            if (!wait_phase<true>(bar(B_HPRE_FULL + sl), v & 1, abort_flag, E_HPRE_FULL)) break;
             float hp[N];
 #pragma unroll
             for (int i = 0; i < N; ++i) hp[i] = hpre[(sl * NT + t) * 4 + i];
@@ -542,15 +599,15 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
 // ---------------------------------------------------------------- host side
 struct Plan {
     bool ok = false;
-    int nstage = 0, smem = 0, max_clusters = 0, tmem_cols = 0;
+    int nstage = 0, smem = 0, max_clusters = 0, nchain = 0, tmem_cols = 0;
 };
 
 template <int N>
 int smem_bytes(int ncb, int nstage) {
     using C = Cfg<N>;
     const int KA = N * ncb;
-    int off = KA * C::ATOM_PHI + nstage * KA * NT * 128 + 2 * S * C::RECV_STRIDE * 4 + 2 * NT * 16 +
-              RING * C::M * 4;
+    int off = KA * C::ATOM_PHI + nstage * KA * NT * 128 + NSLOT * S * C::RECV_STRIDE * 4 +
+              NSLOT * NT * 16 + RING * C::M * 4 + 4 * 2 * NT * 16 * 4;
     off = (off + 15) & ~15;
     off += B_COUNT * 8 + 16;
     return off + 1024;   // alignment slack of the dynamic shared-memory base
@@ -589,12 +646,14 @@ Plan make_plan(int ncb) {
         cudaGetLastError();
         return p;
     }
+    const int nchain = N * ncb < MAXCHAIN ? N * ncb : MAXCHAIN;   // chains that receive MMAs
     int cols = 32;
-    while (cols < ns * NT) cols <<= 1;
+    while (cols < NACC * nchain * NT) cols <<= 1;     // <= 256: two CTAs per SM never block
     p.ok = true;
     p.nstage = ns;
     p.smem = smem;
     p.max_clusters = nc;
+    p.nchain = nchain;
     p.tmem_cols = cols;
     return p;
 }
@@ -668,7 +727,8 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p, int ncb) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, pre_cluster_tc_kernel<N>, map, a.phi, a.b_pre, a.b_post, a.b_res,
                               a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps, a.t_max,
-                              static_cast<__nv_bfloat16*>(a.x_in), a.H, ncb, p.nstage, p.tmem_cols);
+                              static_cast<__nv_bfloat16*>(a.x_in), a.H, ncb, p.nstage, p.nchain,
+                              p.tmem_cols);
 }
 
 }  // namespace tc
