@@ -261,11 +261,13 @@ def run_ours(args, rank, world, local_rank):
     H = torch.empty(T, w.m, dtype=torch.float32, device=dev)
     Y = torch.empty_like(X)
     s = w.scalars()
-    path = mhc.mhc_pre_path_for(T, n, d, tdt)
+    req = {"auto": mhc.PRE_AUTO, "generic": mhc.PRE_GENERIC,
+           "cluster_tc": mhc.PRE_CLUSTER_TC}[args.pre_path]
+    path = mhc.mhc_pre_path_for(T, n, d, tdt) if req == mhc.PRE_AUTO else req
 
     def pre():
-        mhc.mhc_pre(X, phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
-                    s["alpha_res"], s["eps"], s["t_max"], x_in, H)
+        mhc.mhc_pre_with_path(X, phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
+                              s["alpha_res"], s["eps"], s["t_max"], x_in, H, path=req)
 
     def post():
         mhc.mhc_post(X, F, H, Y)
@@ -311,7 +313,7 @@ def run_ours(args, rank, world, local_rank):
                     "gbs": by_pre * T / (pre_ms / 1e3) / 1e9,
                     "path": {1: "generic", 2: "cluster_tc"}.get(path, str(path)),
                     "source": "mhc_hyper_connections_b200/csrc/" +
-                              ("pre_cluster_tc.cu" if path == 2 else "pre_generic.cu")},
+                              {2: "pre_cluster_tc.cu"}.get(path, "pre_generic.cu")},
             "post": {"ms": post_ms, "bytes_per_launch": by_post * T,
                      "gbs": by_post * T / (post_ms / 1e3) / 1e9,
                      "source": "mhc_hyper_connections_b200/csrc/post.cu"}}
@@ -402,6 +404,9 @@ def main():
     ap.add_argument("--config", default=wl.HEADLINE, choices=sorted(wl.CONFIGS))
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the workload (smaller cases for profiling)")
+    ap.add_argument("--pre-path", default="auto",
+                    choices=["auto", "generic", "cluster_tc"],
+                    help="kernel path of the pre stage (default: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -77,7 +77,7 @@ typedef enum {
     MHC_PRE_AUTO = 0,          /* the fastest path that supports the problem          */
     MHC_PRE_GENERIC = 1,       /* CUDA-core kernel: any n <= 8, any d, f32 or bf16    */
     MHC_PRE_CLUSTER_TC = 2     /* thread-block-cluster tensor-core kernel (bf16,      */
-                               /* n <= 4, d in {1024,2048,3072,4096}; see mhc_pre_path)*/
+                               /* n <= 4, d in {1024, 2048, 3072, 4096}; sm_100)      */
 } mhc_pre_path;
 
 /*
@@ -113,9 +113,9 @@ mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre
                              mhc_stream_t stream, mhc_pre_path path);
 
 /*
- * mhc_pre_path -- the path MHC_PRE_AUTO would take for this problem on the current
- * device (host-side query; launches nothing).  Returns MHC_PRE_GENERIC or
- * MHC_PRE_CLUSTER_TC.
+ * mhc_pre_path_for -- the path MHC_PRE_AUTO would take for this problem on the current
+ * device (host-side query; launches nothing): MHC_PRE_CLUSTER_TC where it runs, else
+ * MHC_PRE_GENERIC.
  */
 mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt);
 

@@ -190,7 +190,7 @@ def mhc_device_status() -> int:
 
 
 def mhc_pre_path_for(T: int, n: int, d: int, dtype) -> int:
-    """Kernel path mhc_pre would take on the current device (PRE_GENERIC / PRE_CLUSTER_TC)."""
+    """Kernel path mhc_pre would take on the current device (PRE_GENERIC or PRE_CLUSTER_TC)."""
     import torch
     dt = dtype if isinstance(dtype, int) else (MHC_BF16 if dtype == torch.bfloat16 else MHC_F32)
     return int(load_library().mhc_pre_path_for(int(T), int(n), int(d), dt))

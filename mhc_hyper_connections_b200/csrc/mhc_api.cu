@@ -113,9 +113,9 @@ PreArgs make_pre(const void* X, const float* phi, const float* b_pre, const floa
 extern "C" {
 
 mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
-    if (check_shape(T, n, d, dt) == MHC_OK &&
-        pre_cluster_tc_shape_ok(T, n, d, dt == MHC_BF16 ? BF16 : F32) && pre_cluster_tc_device_ok(n, d))
-        return MHC_PRE_CLUSTER_TC;
+    if (check_shape(T, n, d, dt) != MHC_OK) return MHC_PRE_GENERIC;
+    const DType t = dt == MHC_BF16 ? BF16 : F32;
+    if (pre_cluster_tc_shape_ok(T, n, d, t) && pre_cluster_tc_device_ok(n, d)) return MHC_PRE_CLUSTER_TC;
     return MHC_PRE_GENERIC;
 }
 

@@ -10,27 +10,29 @@
 //     phi_hi = bf16(phi) and phi_lo = bf16(phi - phi_hi) (16 significant bits, above the
 //     TF32 the mixed-precision table asks for), stacked as the 2m rows of the MMA's A
 //     operand (K-major, 128-byte swizzle).
-//   * Tokens stream through in tiles of NT = 16: TMA copies each CTA's slice of the
-//     tile's rows (X read from HBM exactly once) into a ring of shared-memory stages.
-//   * One thread issues tcgen05.mma (M = 64 >= 2m, N = 16 tokens, K = 16) over the
-//     CTA's K-slice into a TMEM accumulator: the partial projection of 16 tokens.
-//   * Partials go to the token's owner CTA (token t of a tile -> CTA t) by st.async
-//     into its shared memory, with the partial sum of squares; the owner adds the 16
-//     partials in a fixed order (deterministic, no atomics -- the property the paper's
-//     deterministic split-k kernel provides), applies 1/r (RMSNorm after the
-//     projection), forms H_pre and broadcasts it to the 16 CTAs.
-//   * Every CTA then computes x_in for its channels from the X tile still in shared
-//     memory and stores it.  Sinkhorn (H_res) and H_post run off the critical path in a
-//     separate warp, 32 tokens at a time, and write the coefficient block H.
+//   * Tokens stream through in tiles of NT = 16: one 4-D TMA box per tile copies the
+//     CTA's slice of the tile (X read from HBM exactly once) into a ring of stages,
+//     ordered as 64-channel atoms a = cb * n + i (channel block cb, stream i).
+//   * Six warps issue tcgen05.mma (M = 64 >= 2m, N = 16 tokens, K = 16) over the CTA's
+//     K-slice, each into its own TMEM accumulator (the tensor core retires one of these
+//     MMAs every ~23 cycles; one issuing warp manages one per ~55).
+//   * Four warps copy every stage into TMEM (a ring of stash slots next to the
+//     accumulators) while adding the tokens' squares, so a stage is free again as soon
+//     as its MMAs are done -- it does not wait for the cluster-wide reduction.
+//   * The epilogue ships each token's partial projection to the token's owner CTA
+//     (token t of a tile -> CTA t) with one bulk shared-to-peer copy per owner; the
+//     owner adds the 16 partials in a fixed order (deterministic, no atomics -- the
+//     property the paper's deterministic split-k kernel provides), applies 1/r (RMSNorm
+//     after the projection), forms H_pre and sends it to the 16 CTAs.  Sinkhorn (H_res)
+//     and H_post run off the critical path in a separate warp, 32 tokens at a time.
+//   * A few tiles later the stash warps read their X back from TMEM and form x_in for
+//     their channels once H_pre has arrived.
 //
-// Warp roles (512 threads): 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2 owner
-// reduction, 3 Sinkhorn / H writer, 4-7 TMEM epilogue, 8-11 sum of squares, 12-15 x_in.
-// Issuing a tcgen05.mma costs the issuing thread ~100 cycles whatever the shape, so four
-// warps issue a tile's MMAs, each into its own TMEM accumulator; the epilogue adds the
-// accumulators in a fixed order and ships each owner its rows with one bulk
-// shared-to-shared copy.
-// Every wait on an mbarrier is bounded in time; on expiry the kernel records the failing
-// wait in a status word, drains its own copies in flight, frees TMEM and returns.
+// Warp roles (544 threads): 0 TMA producer, 1 and 12-16 MMA issuers (warp 1 owns TMEM),
+// 2 owner reduction, 3 Sinkhorn / H writer, 4-7 TMEM epilogue, 8-11 stash / sum of
+// squares / x_in.  Every wait on an mbarrier is bounded in time; on expiry the kernel
+// records the failing wait in a status word, drains its own copies in flight, frees
+// TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,6 +40,7 @@
 
 #include "common.cuh"
 #include "launch.cuh"
+#include "tc_ptx.cuh"
 
 namespace mhc {
 
@@ -50,13 +53,17 @@ namespace tc {
 constexpr int S = 16;          // CTAs per cluster
 constexpr int NT = 16;         // tokens per tile (MMA N)
 constexpr int MAXST = 8;       // max shared-memory stages
-constexpr int NMMA = 4;        // warps issuing tcgen05.mma (issue cost is per thread)
-constexpr int THREADS = 512 + 32 * (NMMA - 1);
-constexpr int NSLOT = 4;       // depth of the cross-CTA rings (partials in, H_pre out)
+constexpr int NMMA = 6;        // MMA-issuing warps = accumulators per buffer
 constexpr int NACC = 2;        // TMEM accumulator buffers (tile k uses buffer k % NACC)
-constexpr int MAXCHAIN = NMMA; // one accumulation chain per MMA warp
+constexpr int NSLOT_P = 4;     // receive ring depth (partials in)
+constexpr int NSLOT_H = 8;     // H_pre ring depth (must exceed the stash lag)
+constexpr int MAXSTASH = 8;    // TMEM stash slots (lag = slots - 1 <= NSLOT_H - 1)
+constexpr int ACC_COLS = NACC * NMMA * NT;   // TMEM columns of accumulators (192)
+constexpr int TMEM_COLS = 512;               // the whole TMEM: one CTA per SM
+constexpr int THREADS = (12 + NMMA - 1) * 32;
 constexpr int RING = 64;       // logits ring (2 batches of 32 tokens)
 constexpr int BATCH = 32;
+constexpr int MIN_SMEM = 120 * 1024;          // keeps a second CTA off the SM (TMEM)
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait, then give up
 
 template <int N>
@@ -78,151 +85,20 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >
 
 // barrier slots (8 bytes each) inside the barrier block
 enum : int {
-    B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = 3 * MAXST,
-    B_PART_FULL = 4 * MAXST, B_PART_EMPTY = B_PART_FULL + NSLOT,
-    B_HPRE_FULL = B_PART_EMPTY + NSLOT, B_HPRE_EMPTY = B_HPRE_FULL + NSLOT,
-    B_LG_FULL = B_HPRE_EMPTY + NSLOT, B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
+    B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = B_ACCF + NACC,
+    B_PART_FULL = B_ACCE + NACC, B_PART_EMPTY = B_PART_FULL + NSLOT_P,
+    B_HPRE_FULL = B_PART_EMPTY + NSLOT_P, B_HPRE_EMPTY = B_HPRE_FULL + NSLOT_H,
+    B_LG_FULL = B_HPRE_EMPTY + NSLOT_H, B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
 };
 
 // status codes: which wait expired
 enum : unsigned {
     E_EMPTY = 1u, E_FULL_MMA = 2u, E_ACCE = 4u, E_ACCF = 8u, E_PART_EMPTY = 16u, E_FULL_SS = 32u,
-    E_PART_FULL = 64u, E_HPRE_EMPTY = 128u, E_FULL_XIN = 256u, E_HPRE_FULL = 512u,
+    E_PART_FULL = 64u, E_HPRE_EMPTY = 128u, E_HPRE_FULL = 512u,
     E_LG_EMPTY = 1024u, E_LG_FULL = 2048u, E_DRAIN = 4096u
 };
 
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r; asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r)); return r;
-}
-__device__ __forceinline__ uint32_t cluster_idx() {
-    uint32_t r; asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r)); return r;
-}
-__device__ __forceinline__ uint32_t cluster_count() {
-    uint32_t r; asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r)); return r;
-}
-__device__ __forceinline__ uint64_t gtimer() {
-    uint64_t t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)); return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).  Used
-// only to say "this buffer may be overwritten": every value read from the buffer has
-// been consumed by an instruction before the arrive, so no release fence is needed (a
-// release here would also wait for this warp's earlier global stores).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cbar) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" :: "r"(cbar) : "memory");
-}
-// CTA-scope acquire: barriers completed by this CTA's own threads, TMA or tensor cores
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-// cluster-scope acquire: barriers whose phase completes with data st.async'd by peers
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_async_v4(uint32_t raddr, float a, float b, float c, float d,
-                                            uint32_t rbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-                 :: "r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar) : "memory");
-}
-__device__ __forceinline__ void st_async_f32(uint32_t raddr, float a, uint32_t rbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];"
-                 :: "r"(raddr), "f"(a), "r"(rbar) : "memory");
-}
-// bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into a peer's,
-// completing `bytes` of transaction count on the peer's mbarrier
-__device__ __forceinline__ void bulk_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                             uint32_t rbar) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(dst_cluster), "r"(src_cta), "r"(bytes), "r"(rbar) : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_allbut1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-                 " [%0], [%1, {%2, %3, %4}], [%5];"
-                 :: "r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 :: "r"(dst_smem), "r"(ncols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t accumulate) {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(IDESC), "r"(accumulate) : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 :: "r"(bar) : "memory");
-}
-// 32 lanes x 16 consecutive 32-bit columns; waits for the load before returning
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
-                 "tcgen05.wait::ld.sync.aligned;"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr) : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// byte offset of 16-byte chunk j of row r inside a 128-byte-swizzled block of 8-row groups
-__device__ __forceinline__ uint32_t sw128_off(int r, int j) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
-}
+using namespace ptx;
 
 // Bounded wait: true when the phase completed; false when the CTA is aborting or the
 // wait expired (then the status word and the CTA's abort flag are set).
@@ -250,7 +126,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                       const float* __restrict__ b_pre, const float* __restrict__ b_post,
                       const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                       int T, int d, float eps, int t_max, __nv_bfloat16* __restrict__ x_in,
-                      float* __restrict__ H, int ncb, int nstage, int nchain, int tmem_cols)
+                      float* __restrict__ H, int ncb, int nstage)
 {
     using C = Cfg<N>;
     constexpr int M = C::M;
@@ -261,6 +137,10 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
 
     const int KA = N * ncb;                 // 64-wide K atoms per CTA (stream x channel block)
     const int cpc = ncb * 64;               // channels per CTA
+    const int nchain = KA < NMMA ? KA : NMMA;          // accumulators that receive MMAs
+    const int stash_cols = 4 * KA;                     // TMEM columns one tile occupies
+    const int nstash = min(MAXSTASH, (TMEM_COLS - ACC_COLS) / stash_cols);
+    const int lag = nstash - 1;                        // x_in trails the stash by `lag` tiles
     const uint32_t stage_bytes = (uint32_t)KA * (NT * 128);
     const uint32_t rank = cluster_ctarank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -269,8 +149,8 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     uint32_t off = 0;
     const uint32_t o_phi = off;  off += (uint32_t)KA * C::ATOM_PHI;
     const uint32_t o_x = off;    off += (uint32_t)nstage * stage_bytes;
-    const uint32_t o_recv = off; off += (uint32_t)NSLOT * S * C::RECV_STRIDE * 4u;
-    const uint32_t o_hpre = off; off += (uint32_t)NSLOT * NT * 16u;
+    const uint32_t o_recv = off; off += (uint32_t)NSLOT_P * S * C::RECV_STRIDE * 4u;
+    const uint32_t o_hpre = off; off += (uint32_t)NSLOT_H * NT * 16u;
     const uint32_t o_ring = off; off += (uint32_t)RING * M * 4u;
     const uint32_t o_stg = off;  off += 4u * 2u * NT * 16u * 4u;     // epilogue staging, per warp x2
     off = (off + 15u) & ~15u;
@@ -291,17 +171,19 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
             mbar_init(bar(B_FULL + s), 1);
-            mbar_init(bar(B_EMPTY + s), NMMA + 8);   // MMA warps + 4 sum-of-squares + 4 x_in
+            mbar_init(bar(B_EMPTY + s), NMMA + 4);   // MMA warps' commits + 4 stash warps
         }
         for (int ab = 0; ab < NACC; ++ab) {
             mbar_init(bar(B_ACCF + ab), NMMA);
-            mbar_init(bar(B_ACCE + ab), 4);       // 4 epilogue warps
+            mbar_init(bar(B_ACCE + ab), 4);          // 4 epilogue warps
         }
-        for (int sl = 0; sl < NSLOT; ++sl) {
+        for (int sl = 0; sl < NSLOT_P; ++sl) {
             mbar_init(bar(B_PART_FULL + sl), 1);
-            mbar_init(bar(B_PART_EMPTY + sl), S);        // one arrive per owner CTA
+            mbar_init(bar(B_PART_EMPTY + sl), S);    // one arrive per owner CTA
+        }
+        for (int sl = 0; sl < NSLOT_H; ++sl) {
             mbar_init(bar(B_HPRE_FULL + sl), 1);
-            mbar_init(bar(B_HPRE_EMPTY + sl), S * 4);    // 4 x_in warps of every CTA
+            mbar_init(bar(B_HPRE_EMPTY + sl), S * 4);   // 4 stash warps of every CTA
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_LG_FULL + b), 1);
@@ -310,12 +192,12 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), (uint32_t)tmem_cols);
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), (uint32_t)TMEM_COLS);
 
     // phi slice -> shared memory as [phi_hi^T ; phi_lo^T] atoms (rows = output columns)
     for (int idx = warp; idx < KA * 8; idx += THREADS / 32) {
         const int a = idx >> 3, j8 = idx & 7;
-        const int i = a / ncb, cb = a - i * ncb;
+        const int cb = a / N, i = a - cb * N;              // atom a = cb * n + i
         const int64_t k0 = (int64_t)i * d + (int64_t)rank * cpc + cb * 64 + j8 * 8;
         if (lane < M) {
             float hi[8], lo[8];
@@ -334,10 +216,8 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int sl = 0; sl < NSLOT; ++sl) {
-            mbar_arrive_tx(bar(B_PART_FULL + sl), C::TX_PART);
-            mbar_arrive_tx(bar(B_HPRE_FULL + sl), C::TX_HPRE);
-        }
+        for (int sl = 0; sl < NSLOT_P; ++sl) mbar_arrive_tx(bar(B_PART_FULL + sl), C::TX_PART);
+        for (int sl = 0; sl < NSLOT_H; ++sl) mbar_arrive_tx(bar(B_HPRE_FULL + sl), C::TX_HPRE);
     }
     tc_fence_before();
     cluster_sync_all();
@@ -355,12 +235,9 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                 if (!wait_phase(bar(B_EMPTY + s), (u & 1) ^ 1, abort_flag, E_EMPTY)) break;
                 mbar_arrive_tx(bar(B_FULL + s), stage_bytes);
                 const int t0 = (cid + k * ncl) * NT;
-                const uint32_t dst = base + o_x + (uint32_t)s * stage_bytes;
-                for (int a = 0; a < KA; ++a) {
-                    const int i = a / ncb, cb = a - i * ncb;
-                    tma_load_3d(dst + (uint32_t)a * (NT * 128), &tmap_x, bar(B_FULL + s),
-                                (int)rank * cpc + cb * 64, i, t0);
-                }
+                // box (64 channels, 16 tokens, n streams, ncb blocks): atoms a = cb * n + i
+                tma_load_4d(base + o_x + (uint32_t)s * stage_bytes, &tmap_x, bar(B_FULL + s),
+                            0, t0, 0, (int)rank * ncb);
                 issued = k + 1;
             }
             // drain: every issued copy has landed before the CTA can leave
@@ -368,25 +245,32 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                 wait_phase(bar(B_FULL + k % nstage), (k / nstage) & 1, abort_flag, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 1 || warp >= 16) {
-        // MMA issuers: warp mw issues the K atoms a = mw, mw + nchain, ... into chain mw
-        const int mw = warp == 1 ? 0 : warp - 15;
+    } else if (warp == 1 || warp >= 12) {
+        // MMA issuers: warp mw issues the K atoms a = mw, mw + nchain, ... into accumulator mw
+        const int mw = warp == 1 ? 0 : warp - 11;     // warps 12.. -> 1..
         if (lane == 0) {
             int issued = 0;
+            // descriptors advance by adding to the start-address field (16-byte units)
+            const uint64_t a_step = (uint64_t)((nchain * C::ATOM_PHI) >> 4);
+            const uint64_t b_step = (uint64_t)((nchain * NT * 128) >> 4);
+            const uint64_t a_first = sw128_desc(base + o_phi + (uint32_t)mw * C::ATOM_PHI);
             for (int k = 0; k < my_tiles; ++k) {
                 const int s = k % nstage, u = k / nstage, ab = k % NACC, ua = k / NACC;
                 if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_MMA)) break;
                 if (!wait_phase(bar(B_ACCE + ab), (ua & 1) ^ 1, abort_flag, E_ACCE)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(ab * nchain * NT);
-                const uint32_t xs = base + o_x + (uint32_t)s * stage_bytes;
+                const uint32_t d_tmem = tmem + (uint32_t)((ab * NMMA + mw) * NT);
+                uint64_t ad = a_first;
+                uint64_t bd = sw128_desc(base + o_x + (uint32_t)s * stage_bytes + (uint32_t)mw * (NT * 128));
+                uint32_t accumulate = 0;
                 for (int a = mw; a < KA && mw < nchain; a += nchain) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = sw128_desc(base + o_phi + (uint32_t)a * C::ATOM_PHI + kk * 32);
-                        const uint64_t bd = sw128_desc(xs + (uint32_t)a * (NT * 128) + kk * 32);
-                        mma_bf16(d_tmem + (uint32_t)(mw * NT), ad, bd, (a != mw) || kk);
-                    }
+                    mma_bf16(d_tmem, ad, bd, IDESC, accumulate);
+                    mma_bf16(d_tmem, ad + 2, bd + 2, IDESC, 1);
+                    mma_bf16(d_tmem, ad + 4, bd + 4, IDESC, 1);
+                    mma_bf16(d_tmem, ad + 6, bd + 6, IDESC, 1);
+                    accumulate = 1;
+                    ad += a_step;
+                    bd += b_step;
                 }
                 mma_commit(bar(B_EMPTY + s));
                 mma_commit(bar(B_ACCF + ab));
@@ -401,9 +285,9 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
         // owner: reduce the 16 partials of this CTA's token, broadcast H_pre, queue logits
         const float invK = 1.0f / (float)(N * d);
         for (int k = 0; k < my_tiles; ++k) {
-            const int sl = k % NSLOT, v = k / NSLOT;
-            if (!wait_phase<true>(bar(B_PART_FULL + sl), v & 1, abort_flag, E_PART_FULL)) break;
-            const float* rb = recv + sl * S * C::RECV_STRIDE;
+            const int slp = k % NSLOT_P, vp = k / NSLOT_P, slh = k % NSLOT_H, vh = k / NSLOT_H;
+            if (!wait_phase<true>(bar(B_PART_FULL + slp), vp & 1, abort_flag, E_PART_FULL)) break;
+            const float* rb = recv + slp * S * C::RECV_STRIDE;
             float ss = 0.f;
 #pragma unroll
             for (int src = 0; src < S; ++src) ss += rb[src * C::RECV_STRIDE + C::RECV_D];
@@ -428,15 +312,15 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             for (int i = 0; i < 4; ++i) hv[i] = __shfl_sync(0xffffffffu, hp, i < N ? i : 31);
             __syncwarp();
             // release the receive slot: arm its next phase, then tell the 16 senders
-            if (lane == 0) mbar_arrive_tx(bar(B_PART_FULL + sl), C::TX_PART);
+            if (lane == 0) mbar_arrive_tx(bar(B_PART_FULL + slp), C::TX_PART);
             __syncwarp();
-            if (lane < S) mbar_arrive_remote(mapa(bar(B_PART_EMPTY + sl), lane));
-            // H_pre of this token -> slot sl of every CTA
-            if (!wait_phase(bar(B_HPRE_EMPTY + sl), (v & 1) ^ 1, abort_flag, E_HPRE_EMPTY)) break;
+            if (lane < S) mbar_arrive_remote(mapa(bar(B_PART_EMPTY + slp), lane));
+            // H_pre of this token -> slot slh of every CTA
+            if (!wait_phase(bar(B_HPRE_EMPTY + slh), (vh & 1) ^ 1, abort_flag, E_HPRE_EMPTY)) break;
             if (lane < S) {
-                const uint32_t dst = smem_u32(hpre + (sl * NT + (int)rank) * 4);
+                const uint32_t dst = smem_u32(hpre + (slh * NT + (int)rank) * 4);
                 st_async_v4(mapa(dst, lane), hv[0], N > 1 ? hv[1] : 0.f, N > 2 ? hv[2] : 0.f,
-                            N > 3 ? hv[3] : 0.f, mapa(bar(B_HPRE_FULL + sl), lane));
+                            N > 3 ? hv[3] : 0.f, mapa(bar(B_HPRE_FULL + slh), lane));
             }
             // [H_pre | res logits | post logits] -> ring for the Sinkhorn warp
             const int bi = k / BATCH, b = bi & 1;
@@ -480,25 +364,34 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             if (lane == 0) mbar_arrive(bar(B_LG_EMPTY + b));
         }
     } else if (warp < 8) {
-        // TMEM epilogue: sum the accumulation chains, stage this warp's 16 rows of the
-        // tile's partial projections, and bulk-copy token t's rows to owner CTA t
+        // TMEM epilogue: sum the accumulators, stage this warp's 16 rows of the tile's
+        // partial projections, and bulk-copy token t's rows to owner CTA t
         const int q = warp & 3;
         const bool has_rows = 16 * q < C::RECV_D;
         const uint32_t nbytes = (uint32_t)min(16, C::RECV_D - 16 * q) * 4u;
         float* stg = reinterpret_cast<float*>(sb + o_stg) + q * (2 * NT * 16);
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         for (int k = 0; k < my_tiles; ++k) {
-            const int ab = k % NACC, ua = k / NACC, sl = k % NSLOT, v = k / NSLOT;
+            const int ab = k % NACC, ua = k / NACC, slp = k % NSLOT_P, vp = k / NSLOT_P;
             if (!wait_phase(bar(B_ACCF + ab), ua & 1, abort_flag, E_ACCF)) break;
             tc_fence_after();
             float dv[16];
             if (has_rows) {
-                tmem_ld16(tq + (uint32_t)(ab * nchain * NT), dv);
-                for (int c = 1; c < nchain; ++c) {
-                    float e[16];
-                    tmem_ld16(tq + (uint32_t)((ab * nchain + c) * NT), e);
+                // accumulators are adjacent 16-column blocks: load two per instruction
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) dv[t] += e[t];
+                for (int t = 0; t < NT; ++t) dv[t] = 0.f;
+                for (int c = 0; c < nchain; c += 2) {
+                    if (c + 1 < nchain) {
+                        float e[32];
+                        tmem_ld32(tq + (uint32_t)((ab * NMMA + c) * NT), e);
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) dv[t] += e[t] + e[NT + t];
+                    } else {
+                        float e[16];
+                        tmem_ld16(tq + (uint32_t)((ab * NMMA + c) * NT), e);
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) dv[t] += e[t];
+                    }
                 }
             }
             tc_fence_before();
@@ -514,76 +407,88 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (!wait_phase(bar(B_PART_EMPTY + sl), (v & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
+            if (!wait_phase(bar(B_PART_EMPTY + slp), (vp & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
             if (lane < NT) {
                 const uint32_t dst = base + o_recv +
-                                     (uint32_t)((sl * S + (int)rank) * C::RECV_STRIDE + 16 * q) * 4u;
+                                     (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE + 16 * q) * 4u;
                 bulk_to_peer(mapa(dst, lane), smem_u32(sbuf + lane * 16), nbytes,
-                             mapa(bar(B_PART_FULL + sl), lane));
+                             mapa(bar(B_PART_FULL + slp), lane));
             }
         }
         if (lane < NT) bulk_wait_all();
-    } else if (warp < 12) {
-        // sum of squares of this CTA's slice of every token of the tile -> owners
-        const int t = (warp - 8) * 4 + (lane >> 3), u8 = lane & 7;
-        for (int k = 0; k < my_tiles; ++k) {
-            const int s = k % nstage, u = k / nstage, sl = k % NSLOT, v = k / NSLOT;
-            if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_SS)) break;
-            const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
-            float ss = 0.f;
-            for (int a = 0; a < KA; ++a) {
-                const uint4 w = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + sw128_off(t, u8));
-                float f[8];
-                Vec16<__nv_bfloat16>::unpack(w, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-            }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
-            if (!wait_phase(bar(B_PART_EMPTY + sl), (v & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
-            if (u8 == 0) {
-                const uint32_t dst = base + o_recv +
-                                     (uint32_t)((sl * S + (int)rank) * C::RECV_STRIDE + C::RECV_D) * 4u;
-                st_async_f32(mapa(dst, t), ss, mapa(bar(B_PART_FULL + sl), t));
-            }
-        }
     } else {
-        // x_in = sum_i H_pre[i] X_i for this CTA's channels, from the tile in shared memory
-        const int t = (warp - 12) * 4 + (lane >> 3), u8 = lane & 7;
-        const int coff = (int)rank * cpc + (u8 << 3);
-        for (int k = 0; k < my_tiles; ++k) {
-            const int s = k % nstage, u = k / nstage, sl = k % NSLOT, v = k / NSLOT;
-            const int64_t tok = (int64_t)(cid + k * ncl) * NT + t;
-            if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_XIN)) break;
-            if (!wait_phase<true>(bar(B_HPRE_FULL + sl), v & 1, abort_flag, E_HPRE_FULL)) break;
+        // stash warps (8-11): thread = (token t, 16-byte chunk u8) = TMEM lane 32q + lane.
+        // Per tile: copy the token's chunk of every atom to TMEM, add its squares, send the
+        // sum to the owner, release the stage; `lag` tiles later form x_in from TMEM.
+        const int q = warp & 3;
+        const int t = q * 4 + (lane >> 3), u8 = lane & 7;
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        auto stash_col = [&](int k) -> uint32_t { return (uint32_t)(ACC_COLS + (k % nstash) * stash_cols); };
+        auto read_map = [&](int j) -> bool {     // x_in for tile j
+            const int slh = j % NSLOT_H, vh = j / NSLOT_H;
+            if (!wait_phase<true>(bar(B_HPRE_FULL + slh), vh & 1, abort_flag, E_HPRE_FULL)) return false;
             float hp[N];
 #pragma unroll
-            for (int i = 0; i < N; ++i) hp[i] = hpre[(sl * NT + t) * 4 + i];
-            const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
+            for (int i = 0; i < N; ++i) hp[i] = hpre[(slh * NT + t) * 4 + i];
+            __syncwarp();
+            // arm the slot's next phase: it cannot complete before all four stash warps of
+            // every CTA (this one's included) have released this phase below
+            if (warp == 8 && lane == 0) mbar_arrive_tx(bar(B_HPRE_FULL + slh), C::TX_HPRE);
+            __syncwarp();
+            if (lane < S) mbar_arrive_remote(mapa(bar(B_HPRE_EMPTY + slh), lane));
+            const int64_t tok = (int64_t)(cid + j * ncl) * NT + t;
+            const uint32_t col = tq + stash_col(j);
             for (int cb = 0; cb < ncb; ++cb) {
                 float acc[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
                 for (int i = 0; i < N; ++i) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(
-                        xs + (i * ncb + cb) * (NT * 128) + sw128_off(t, u8));
+                    const uint4 w = tmem_ld4(col + (uint32_t)(4 * (cb * N + i)));
                     float f[8];
                     Vec16<__nv_bfloat16>::unpack(w, f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) acc[e] = fmaf(hp[i], f[e], acc[e]);
                 }
-                if (tok < T) st_v4(x_in + tok * d + coff + cb * 64, Vec16<__nv_bfloat16>::pack(acc));
+                if (tok < T)
+                    st_v4(x_in + tok * d + (int)rank * cpc + cb * 64 + u8 * 8, Vec16<__nv_bfloat16>::pack(acc));
             }
+            return true;
+        };
+        bool ok = true;
+        int done = 0;                         // tiles whose x_in has been formed
+        for (int k = 0; k < my_tiles && ok; ++k) {
+            const int s = k % nstage, u = k / nstage, slp = k % NSLOT_P, vp = k / NSLOT_P;
+            if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_SS)) break;
+            const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
+            const uint32_t col = tq + stash_col(k);
+            float ss = 0.f;
+            for (int a = 0; a < KA; ++a) {
+                const uint4 w = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + sw128_off(t, u8));
+                tmem_st4(col + (uint32_t)(4 * a), w);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(w, f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            }
+            tmem_wait_st();
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 4);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
-            if (warp == 12 && lane == 0) mbar_arrive_tx(bar(B_HPRE_FULL + sl), C::TX_HPRE);
-            __syncwarp();
-            if (lane < S) mbar_arrive_remote(mapa(bar(B_HPRE_EMPTY + sl), lane));
+            if (!wait_phase(bar(B_PART_EMPTY + slp), (vp & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
+            if (u8 == 0) {
+                const uint32_t dst = base + o_recv +
+                                     (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE + C::RECV_D) * 4u;
+                st_async_f32(mapa(dst, t), ss, mapa(bar(B_PART_FULL + slp), t));
+            }
+            if (k >= lag) {
+                ok = read_map(k - lag);
+                done = k - lag + 1;
+            }
         }
+        for (int j = done; j < my_tiles && ok && !*abort_flag; ++j) ok = read_map(j);
     }
 
     // ---------------- tear-down: no peer touches this CTA's shared memory after this
@@ -592,25 +497,26 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)tmem_cols);
+        tmem_dealloc(tmem, (uint32_t)TMEM_COLS);
     }
 }
 
 // ---------------------------------------------------------------- host side
 struct Plan {
     bool ok = false;
-    int nstage = 0, smem = 0, max_clusters = 0, nchain = 0, tmem_cols = 0;
+    int nstage = 0, smem = 0, max_clusters = 0;
 };
 
 template <int N>
 int smem_bytes(int ncb, int nstage) {
     using C = Cfg<N>;
     const int KA = N * ncb;
-    int off = KA * C::ATOM_PHI + nstage * KA * NT * 128 + NSLOT * S * C::RECV_STRIDE * 4 +
-              NSLOT * NT * 16 + RING * C::M * 4 + 4 * 2 * NT * 16 * 4;
+    int off = KA * C::ATOM_PHI + nstage * KA * NT * 128 + NSLOT_P * S * C::RECV_STRIDE * 4 +
+              NSLOT_H * NT * 16 + RING * C::M * 4 + 4 * 2 * NT * 16 * 4;
     off = (off + 15) & ~15;
     off += B_COUNT * 8 + 16;
-    return off + 1024;   // alignment slack of the dynamic shared-memory base
+    off += 1024;         // alignment slack of the dynamic shared-memory base
+    return off < MIN_SMEM ? MIN_SMEM : off;
 }
 
 template <int N>
@@ -646,15 +552,10 @@ Plan make_plan(int ncb) {
         cudaGetLastError();
         return p;
     }
-    const int nchain = N * ncb < MAXCHAIN ? N * ncb : MAXCHAIN;   // chains that receive MMAs
-    int cols = 32;
-    while (cols < NACC * nchain * NT) cols <<= 1;     // <= 256: two CTAs per SM never block
     p.ok = true;
     p.nstage = ns;
     p.smem = smem;
     p.max_clusters = nc;
-    p.nchain = nchain;
-    p.tmem_cols = cols;
     return p;
 }
 
@@ -699,15 +600,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int N>
 cudaError_t launch_n(const PreArgs& a, const Plan& p, int ncb) {
-    // X viewed as 3-D: (channel c: d, stream i: n, token t: T); box = 64 channels x 1 x 16 tokens
+    // X viewed as 4-D: (channel within a 64-block: 64, token: T, stream: n, block: d/64);
+    // one box (64, 16, n, d/1024) is a CTA's whole slice of a 16-token tile
     CUtensorMap map;
-    const cuuint64_t dims[3] = {(cuuint64_t)a.d, (cuuint64_t)N, (cuuint64_t)a.T};
-    const cuuint64_t strides[2] = {(cuuint64_t)a.d * 2, (cuuint64_t)N * a.d * 2};
-    const cuuint32_t box[3] = {64, 1, NT};
-    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint64_t dims[4] = {64, (cuuint64_t)a.T, (cuuint64_t)N, (cuuint64_t)(a.d / 64)};
+    const cuuint64_t strides[3] = {(cuuint64_t)N * a.d * 2, (cuuint64_t)a.d * 2, 128};
+    const cuuint32_t box[4] = {64, NT, (cuuint32_t)N, (cuuint32_t)ncb};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
     auto enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides,
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.X), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -727,8 +629,7 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p, int ncb) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, pre_cluster_tc_kernel<N>, map, a.phi, a.b_pre, a.b_post, a.b_res,
                               a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps, a.t_max,
-                              static_cast<__nv_bfloat16*>(a.x_in), a.H, ncb, p.nstage, p.nchain,
-                              p.tmem_cols);
+                              static_cast<__nv_bfloat16*>(a.x_in), a.H, ncb, p.nstage);
 }
 
 }  // namespace tc
