@@ -1,0 +1,37 @@
+"""Multi-GPU plumbing for the data-parallel forward path.
+
+Tokens are independent in both mHC stages, so the forward path shards the token axis:
+each rank runs the pre and post stages on its own contiguous block of tokens, and no
+collective touches the data path.  The helpers here split the token axis and combine
+per-rank timings (the job is as slow as its slowest rank).  They work with any
+torch.distributed backend (NCCL on GPUs, gloo in the CPU tests).
+"""
+from __future__ import annotations
+
+
+def token_shard(T_total: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous [start, stop) block of tokens for `rank`; blocks differ by at most one."""
+    if world < 1 or not 0 <= rank < world or T_total < 0:
+        raise ValueError("bad shard request")
+    base, extra = divmod(T_total, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of `value` over all ranks of the default process group (the value itself when
+    torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    if max_ms <= 0:
+        raise ValueError("time must be positive")
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
