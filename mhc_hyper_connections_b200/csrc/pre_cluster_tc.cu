@@ -25,12 +25,12 @@
 //     property the paper's deterministic split-k kernel provides), applies 1/r (RMSNorm
 //     after the projection), forms H_pre and sends it to the 16 CTAs.  Sinkhorn (H_res)
 //     and H_post run off the critical path in a separate warp, 32 tokens at a time.
-//   * A few tiles later the stash warps read their X back from TMEM and form x_in for
-//     their channels once H_pre has arrived.
+//   * Once a tile's H_pre has arrived, four x_in warps read the tile back from TMEM and
+//     form x_in for their channels.
 //
-// Warp roles (544 threads): 0 TMA producer, 1 and 12-16 MMA issuers (warp 1 owns TMEM),
-// 2 owner reduction, 3 Sinkhorn / H writer, 4-7 TMEM epilogue, 8-11 stash / sum of
-// squares / x_in.  Every wait on an mbarrier is bounded in time; on expiry the kernel
+// Warp roles (672 threads): 0 TMA producer, 1 and 16-20 MMA issuers (warp 1 owns TMEM),
+// 2 owner reduction, 3 Sinkhorn / H writer, 4-7 TMEM epilogue, 8-11 stash and sums of
+// squares, 12-15 x_in (same TMEM lane quarters as the stash warps).  Every wait on an mbarrier is bounded in time; on expiry the kernel
 // records the failing wait in a status word, drains its own copies in flight, frees
 // TMEM and returns.
 #include <cuda.h>
@@ -56,11 +56,11 @@ constexpr int MAXST = 8;       // max shared-memory stages
 constexpr int NMMA = 6;        // MMA-issuing warps = accumulators per buffer
 constexpr int NACC = 2;        // TMEM accumulator buffers (tile k uses buffer k % NACC)
 constexpr int NSLOT_P = 4;     // receive ring depth (partials in)
-constexpr int NSLOT_H = 8;     // H_pre ring depth (must exceed the stash lag)
-constexpr int MAXSTASH = 8;    // TMEM stash slots (lag = slots - 1 <= NSLOT_H - 1)
+constexpr int NSLOT_H = 8;     // H_pre ring depth
+constexpr int MAXSTASH = 8;    // TMEM stash slots (tiles of X held for x_in)
 constexpr int ACC_COLS = NACC * NMMA * NT;   // TMEM columns of accumulators (192)
 constexpr int TMEM_COLS = 512;               // the whole TMEM: one CTA per SM
-constexpr int THREADS = (12 + NMMA - 1) * 32;
+constexpr int THREADS = (16 + NMMA - 1) * 32;
 constexpr int RING = 64;       // logits ring (2 batches of 32 tokens)
 constexpr int BATCH = 32;
 constexpr int MIN_SMEM = 120 * 1024;          // keeps a second CTA off the SM (TMEM)
@@ -88,14 +88,17 @@ enum : int {
     B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = B_ACCF + NACC,
     B_PART_FULL = B_ACCE + NACC, B_PART_EMPTY = B_PART_FULL + NSLOT_P,
     B_HPRE_FULL = B_PART_EMPTY + NSLOT_P, B_HPRE_EMPTY = B_HPRE_FULL + NSLOT_H,
-    B_LG_FULL = B_HPRE_EMPTY + NSLOT_H, B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
+    B_LG_FULL = B_HPRE_EMPTY + NSLOT_H, B_LG_EMPTY = B_LG_FULL + 2, B_SFULL = B_LG_EMPTY + 2,
+    B_SEMPTY = B_SFULL + MAXSTASH, B_STG_READY = B_SEMPTY + MAXSTASH, B_STG_FREE = B_STG_READY + 2,
+    B_COUNT = B_STG_FREE + 2
 };
 
 // status codes: which wait expired
 enum : unsigned {
     E_EMPTY = 1u, E_FULL_MMA = 2u, E_ACCE = 4u, E_ACCF = 8u, E_PART_EMPTY = 16u, E_FULL_SS = 32u,
     E_PART_FULL = 64u, E_HPRE_EMPTY = 128u, E_HPRE_FULL = 512u,
-    E_LG_EMPTY = 1024u, E_LG_FULL = 2048u, E_DRAIN = 4096u
+    E_LG_EMPTY = 1024u, E_LG_FULL = 2048u, E_DRAIN = 4096u, E_SFULL = 8192u, E_SEMPTY = 16384u,
+    E_STG = 32768u
 };
 
 using namespace ptx;
@@ -140,7 +143,6 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     const int nchain = KA < NMMA ? KA : NMMA;          // accumulators that receive MMAs
     const int stash_cols = 4 * KA;                     // TMEM columns one tile occupies
     const int nstash = min(MAXSTASH, (TMEM_COLS - ACC_COLS) / stash_cols);
-    const int lag = nstash - 1;                        // x_in trails the stash by `lag` tiles
     const uint32_t stage_bytes = (uint32_t)KA * (NT * 128);
     const uint32_t rank = cluster_ctarank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,7 +154,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     const uint32_t o_recv = off; off += (uint32_t)NSLOT_P * S * C::RECV_STRIDE * 4u;
     const uint32_t o_hpre = off; off += (uint32_t)NSLOT_H * NT * 16u;
     const uint32_t o_ring = off; off += (uint32_t)RING * M * 4u;
-    const uint32_t o_stg = off;  off += 4u * 2u * NT * 16u * 4u;     // epilogue staging, per warp x2
+    const uint32_t o_stg = off;  off += 2u * NT * C::RECV_D * 4u;    // epilogue staging, 2 tiles
     off = (off + 15u) & ~15u;
     const uint32_t o_bar = off;  off += B_COUNT * 8u;
     const uint32_t o_misc = off;
@@ -188,6 +190,14 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_LG_FULL + b), 1);
             mbar_init(bar(B_LG_EMPTY + b), 1);
+        }
+        for (int j = 0; j < MAXSTASH; ++j) {
+            mbar_init(bar(B_SFULL + j), 4);      // 4 stash warps wrote the slot
+            mbar_init(bar(B_SEMPTY + j), 4);     // 4 x_in warps read it
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_STG_READY + b), 4);  // 4 epilogue warps staged their rows
+            mbar_init(bar(B_STG_FREE + b), 4);   // 4 epilogue warps' copies have read it
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -245,9 +255,9 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                 wait_phase(bar(B_FULL + k % nstage), (k / nstage) & 1, abort_flag, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 1 || warp >= 12) {
+    } else if (warp == 1 || warp >= 16) {
         // MMA issuers: warp mw issues the K atoms a = mw, mw + nchain, ... into accumulator mw
-        const int mw = warp == 1 ? 0 : warp - 11;     // warps 12.. -> 1..
+        const int mw = warp == 1 ? 0 : warp - 15;     // warps 16.. -> 1..
         if (lane == 0) {
             int issued = 0;
             // descriptors advance by adding to the start-address field (16-byte units)
@@ -284,6 +294,11 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
     } else if (warp == 2) {
         // owner: reduce the 16 partials of this CTA's token, broadcast H_pre, queue logits
         const float invK = 1.0f / (float)(N * d);
+        // lane j's bias and gate scalar, loaded once
+        float bias = 0.f, alpha = 0.f;
+        if (lane < N) { bias = __ldg(b_pre + lane); alpha = a_pre; }
+        else if (lane < N + N * N) { bias = __ldg(b_res + (lane - N)); alpha = a_res; }
+        else if (lane < M) { bias = __ldg(b_post + (lane - N - N * N)); alpha = a_post; }
         for (int k = 0; k < my_tiles; ++k) {
             const int slp = k % NSLOT_P, vp = k / NSLOT_P, slh = k % NSLOT_H, vh = k / NSLOT_H;
             if (!wait_phase<true>(bar(B_PART_FULL + slp), vp & 1, abort_flag, E_PART_FULL)) break;
@@ -302,10 +317,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                 h = hh + hl;
             }
             const float inv_r = 1.0f / sqrtf(ss * invK + eps);
-            float z = 0.f;
-            if (lane < N) z = a_pre * (h * inv_r) + __ldg(b_pre + lane);
-            else if (lane < N + N * N) z = a_res * (h * inv_r) + __ldg(b_res + (lane - N));
-            else if (lane < M) z = a_post * (h * inv_r) + __ldg(b_post + (lane - N - N * N));
+            const float z = alpha * (h * inv_r) + bias;
             const float hp = lane < N ? sigmoid_f32(z) : 0.f;
             float hv[4];
 #pragma unroll
@@ -364,15 +376,16 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             if (lane == 0) mbar_arrive(bar(B_LG_EMPTY + b));
         }
     } else if (warp < 8) {
-        // TMEM epilogue: sum the accumulators, stage this warp's 16 rows of the tile's
-        // partial projections, and bulk-copy token t's rows to owner CTA t
+        // TMEM epilogue: sum the accumulators and stage the tile's partial projections as
+        // [token][row]; then warp q bulk-copies tokens 4q..4q+3 to their owner CTAs (one
+        // copy of the token's whole row each: 16 copies per tile in all)
         const int q = warp & 3;
         const bool has_rows = 16 * q < C::RECV_D;
-        const uint32_t nbytes = (uint32_t)min(16, C::RECV_D - 16 * q) * 4u;
-        float* stg = reinterpret_cast<float*>(sb + o_stg) + q * (2 * NT * 16);
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        float* stg0 = reinterpret_cast<float*>(sb + o_stg);
         for (int k = 0; k < my_tiles; ++k) {
             const int ab = k % NACC, ua = k / NACC, slp = k % NSLOT_P, vp = k / NSLOT_P;
+            const int b = k & 1, ub = k >> 1;
             if (!wait_phase(bar(B_ACCF + ab), ua & 1, abort_flag, E_ACCF)) break;
             tc_fence_after();
             float dv[16];
@@ -397,29 +410,75 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_ACCE + ab));
-            if (!has_rows) continue;
-            float* sbuf = stg + (k & 1) * (NT * 16);
-            if (lane < NT) bulk_wait_read_allbut1();     // copies out of sbuf two tiles ago done
-            __syncwarp();
-            if (lane < 16) {
+            // stage rows 16q..16q+15 of every token into buffer b
+            float* stg = stg0 + b * (NT * C::RECV_D);
+            if (!wait_phase(bar(B_STG_FREE + b), (ub & 1) ^ 1, abort_flag, E_STG)) break;
+            if (has_rows && lane < 16 && 16 * q + lane < C::RECV_D) {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) sbuf[t * 16 + lane] = dv[t];
+                for (int t = 0; t < NT; ++t) stg[t * C::RECV_D + 16 * q + lane] = dv[t];
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_STG_READY + b));
+            if (!wait_phase(bar(B_STG_READY + b), ub & 1, abort_flag, E_STG)) break;
             if (!wait_phase(bar(B_PART_EMPTY + slp), (vp & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
-            if (lane < NT) {
+            if (lane < 4) {
+                const int owner = 4 * q + lane;
+                const uint32_t dst = base + o_recv + (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE) * 4u;
+                bulk_to_peer(mapa(dst, owner), smem_u32(stg + owner * C::RECV_D), C::RECV_D * 4,
+                             mapa(bar(B_PART_FULL + slp), owner));
+                // the previous tile's copies (other buffer) have read their source by now
+                bulk_wait_read_allbut1();
+            }
+            __syncwarp();
+            if (k > 0 && lane == 0) mbar_arrive(bar(B_STG_FREE + (b ^ 1)));
+        }
+        if (lane < 4) bulk_wait_all();
+    } else if (warp < 12) {
+        // stash warps (8-11): thread = (token t, 16-byte chunk u8) = TMEM lane 32q + lane.
+        // Per tile: copy the token's chunk of every atom into a TMEM stash slot, add its
+        // squares, send the sum to the owner and release the stage.
+        const int q = warp & 3;
+        const int t = q * 4 + (lane >> 3), u8 = lane & 7;
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        auto stash_col = [&](int k) -> uint32_t { return (uint32_t)(ACC_COLS + (k % nstash) * stash_cols); };
+        for (int k = 0; k < my_tiles; ++k) {
+            const int s = k % nstage, u = k / nstage, slp = k % NSLOT_P, vp = k / NSLOT_P;
+            const int js = k % nstash, us = k / nstash;
+            if (!wait_phase(bar(B_SEMPTY + js), (us & 1) ^ 1, abort_flag, E_SEMPTY)) break;
+            if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_SS)) break;
+            tc_fence_after();
+            const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
+            const uint32_t col = tq + stash_col(k);
+            float ss = 0.f;
+            for (int a = 0; a < KA; ++a) {
+                const uint4 w = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + sw128_off(t, u8));
+                tmem_st4(col + (uint32_t)(4 * a), w);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(w, f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(B_EMPTY + s));
+                mbar_arrive(bar(B_SFULL + js));
+            }
+            if (!wait_phase(bar(B_PART_EMPTY + slp), (vp & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
+            if (u8 == 0) {
                 const uint32_t dst = base + o_recv +
-                                     (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE + 16 * q) * 4u;
-                bulk_to_peer(mapa(dst, lane), smem_u32(sbuf + lane * 16), nbytes,
-                             mapa(bar(B_PART_FULL + slp), lane));
+                                     (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE + C::RECV_D) * 4u;
+                st_async_f32(mapa(dst, t), ss, mapa(bar(B_PART_FULL + slp), t));
             }
         }
-        if (lane < NT) bulk_wait_all();
     } else {
-        // stash warps (8-11): thread = (token t, 16-byte chunk u8) = TMEM lane 32q + lane.
-        // Per tile: copy the token's chunk of every atom to TMEM, add its squares, send the
-        // sum to the owner, release the stage; `lag` tiles later form x_in from TMEM.
+        // x_in warps (12-15), same TMEM lanes as the stash warps: once a tile's H_pre has
+        // arrived, read its stash slot back and form x_in for this CTA's channels
         const int q = warp & 3;
         const int t = q * 4 + (lane >> 3), u8 = lane & 7;
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
@@ -433,11 +492,12 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             __syncwarp();
             // arm the slot's next phase: it cannot complete before all four stash warps of
             // every CTA (this one's included) have released this phase below
-            if (warp == 8 && lane == 0) mbar_arrive_tx(bar(B_HPRE_FULL + slh), C::TX_HPRE);
+            if (warp == 12 && lane == 0) mbar_arrive_tx(bar(B_HPRE_FULL + slh), C::TX_HPRE);
             __syncwarp();
             if (lane < S) mbar_arrive_remote(mapa(bar(B_HPRE_EMPTY + slh), lane));
             const int64_t tok = (int64_t)(cid + j * ncl) * NT + t;
             const uint32_t col = tq + stash_col(j);
+            tc_fence_after();
             for (int cb = 0; cb < ncb; ++cb) {
                 float acc[8];
 #pragma unroll
@@ -455,40 +515,14 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             }
             return true;
         };
-        bool ok = true;
-        int done = 0;                         // tiles whose x_in has been formed
-        for (int k = 0; k < my_tiles && ok; ++k) {
-            const int s = k % nstage, u = k / nstage, slp = k % NSLOT_P, vp = k / NSLOT_P;
-            if (!wait_phase(bar(B_FULL + s), u & 1, abort_flag, E_FULL_SS)) break;
-            const uint8_t* xs = sb + o_x + (uint32_t)s * stage_bytes;
-            const uint32_t col = tq + stash_col(k);
-            float ss = 0.f;
-            for (int a = 0; a < KA; ++a) {
-                const uint4 w = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + sw128_off(t, u8));
-                tmem_st4(col + (uint32_t)(4 * a), w);
-                float f[8];
-                Vec16<__nv_bfloat16>::unpack(w, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-            }
-            tmem_wait_st();
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        for (int j = 0; j < my_tiles; ++j) {
+            const int js = j % nstash, us = j / nstash;
+            if (!wait_phase(bar(B_SFULL + js), us & 1, abort_flag, E_SFULL)) break;
+            if (!read_map(j)) break;
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
-            if (!wait_phase(bar(B_PART_EMPTY + slp), (vp & 1) ^ 1, abort_flag, E_PART_EMPTY)) break;
-            if (u8 == 0) {
-                const uint32_t dst = base + o_recv +
-                                     (uint32_t)((slp * S + (int)rank) * C::RECV_STRIDE + C::RECV_D) * 4u;
-                st_async_f32(mapa(dst, t), ss, mapa(bar(B_PART_FULL + slp), t));
-            }
-            if (k >= lag) {
-                ok = read_map(k - lag);
-                done = k - lag + 1;
-            }
+            if (lane == 0) mbar_arrive(bar(B_SEMPTY + js));
         }
-        for (int j = done; j < my_tiles && ok && !*abort_flag; ++j) ok = read_map(j);
     }
 
     // ---------------- tear-down: no peer touches this CTA's shared memory after this
@@ -512,7 +546,7 @@ int smem_bytes(int ncb, int nstage) {
     using C = Cfg<N>;
     const int KA = N * ncb;
     int off = KA * C::ATOM_PHI + nstage * KA * NT * 128 + NSLOT_P * S * C::RECV_STRIDE * 4 +
-              NSLOT_H * NT * 16 + RING * C::M * 4 + 4 * 2 * NT * 16 * 4;
+              NSLOT_H * NT * 16 + RING * C::M * 4 + 2 * NT * C::RECV_D * 4;
     off = (off + 15) & ~15;
     off += B_COUNT * 8 + 16;
     off += 1024;         // alignment slack of the dynamic shared-memory base
