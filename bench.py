@@ -42,8 +42,9 @@ FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
 # the named kernel on the headline workload, with the sha256 of the kernel source it was
 # measured on; reported as null once that source changes.
 NCU_TRAFFIC = {
-    # pre (cluster tensor-core kernel), measured at T=4096 and scaled x4 to T=16384
-    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((135.8656 + 16.002048) * 4e6), "ad438fd4aa325133"),
+    # measured at T=8192 (X = 256 MiB, twice the L2) and scaled x2 to T=16384
+    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.178304 + 50.199296) * 2e6), "66d4bb37f6ae0b95"),
+    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.358144 + 213.037056) * 2e6), "96dbcd70460419e6"),
 }
 
 

@@ -565,7 +565,9 @@ Plan make_plan(int ncb) {
     if (smem_bytes<N>(ncb, ns) - 1024 < N * ncb * Cfg<N>::ATOM_PHI + (8 - Cfg<N>::G) * 1024) return p;
     const int smem = smem_bytes<N>(ncb, ns);
     auto kern = pre_cluster_tc_kernel<N>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+    // the limit is a property of the function, shared by every plan of this n: set the device's
+    // maximum so that no plan's launch is refused after another plan was made
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
         cudaGetLastError();
         return p;
