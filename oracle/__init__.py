@@ -11,6 +11,10 @@ What each function follows (page title, section / equation):
                  a/b/c-tilde and gate; slavadubrov.com article Eq. 3 (read map).
   * mhc_post  -- slavadubrov.com article, "Kernmechanismen" Eq. 3; the knowledge
                  page's HC update equation.
+  * mhc_projection -- the normalised projection h of the same page's rmsnorm and
+                 projection equations (what the training forward saves for the backward).
+  * mhc_backward -- reverse mode of pre + post (the chain rule through the steps above,
+                 last step first; the Sinkhorn rounds recomputed from the logits).
 
 Parity pins for every function live in tests/test_oracle_pins.py.
 """
@@ -60,6 +64,14 @@ def _load():
             lib.oracle_mhc_post.argtypes = [_dp, _dp, _dp, ctypes.c_long, ctypes.c_int,
                                             ctypes.c_int, _dp, ctypes.c_int]
             lib.oracle_mhc_post.restype = None
+            lib.oracle_mhc_projection.argtypes = [_dp, _dp, ctypes.c_long, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_double, _dp, ctypes.c_int]
+            lib.oracle_mhc_projection.restype = None
+            lib.oracle_mhc_backward.argtypes = ([_dp] * 6 + [ctypes.c_double] * 3 +
+                                                [ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_double, ctypes.c_int] + [_dp] * 9 +
+                                                [ctypes.c_int])
+            lib.oracle_mhc_backward.restype = None
             lib.oracle_threads_used.argtypes = [ctypes.c_int]
             lib.oracle_threads_used.restype = ctypes.c_int
             _lib = lib
@@ -108,6 +120,41 @@ def mhc_post(X, F_out, H, nthreads: int = 1) -> np.ndarray:
     assert F_out.shape == (T, d) and H.shape == (T, n * n + 2 * n)
     out = np.empty_like(X)
     _load().oracle_mhc_post(_p(X), _p(F_out), _p(H), T, n, d, _p(out), int(nthreads))
+    return out
+
+
+def mhc_projection(X, phi, eps: float = 1e-20, nthreads: int = 1) -> np.ndarray:
+    """h = RMSNorm(vec X_t) . phi for every token: X [T, n, d] -> h [T, n*n+2n] in fp64."""
+    X, phi = _c(X), _c(phi)
+    T, n, d = X.shape
+    m = n * n + 2 * n
+    assert phi.shape == (n * d, m), phi.shape
+    h = np.empty((T, m), np.float64)
+    _load().oracle_mhc_projection(_p(X), _p(phi), T, n, d, float(eps), _p(h), int(nthreads))
+    return h
+
+
+def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+                 dX_out, dx_in, eps: float = 1e-20, t_max: int = 20, nthreads: int = 1) -> dict:
+    """Gradients of L = <dX_out, X'> + <dx_in, x_in> with respect to every input of pre +
+    post, in fp64: dict with dX [T,n,d], dF_out [T,d], dphi [n*d,m], db_pre [n],
+    db_post [n], db_res [n,n] and dalpha [3] = (pre, post, res), the alpha arguments' order."""
+    X, F_out, phi = _c(X), _c(F_out), _c(phi)
+    T, n, d = X.shape
+    m = n * n + 2 * n
+    assert F_out.shape == (T, d) and phi.shape == (n * d, m)
+    dX_out, dx_in = _c(dX_out), _c(dx_in)
+    assert dX_out.shape == (T, n, d) and dx_in.shape == (T, d)
+    b_pre, b_post, b_res = _c(b_pre).reshape(n), _c(b_post).reshape(n), _c(b_res).reshape(n * n)
+    out = dict(dX=np.empty((T, n, d)), dF_out=np.empty((T, d)), dphi=np.empty((n * d, m)),
+               db_pre=np.empty(n), db_post=np.empty(n), db_res=np.empty(n * n), dalpha=np.empty(3))
+    _load().oracle_mhc_backward(_p(X), _p(F_out), _p(phi), _p(b_pre), _p(b_post), _p(b_res),
+                                float(alpha_pre), float(alpha_post), float(alpha_res),
+                                T, n, d, float(eps), int(t_max), _p(dX_out), _p(dx_in),
+                                _p(out["dX"]), _p(out["dF_out"]), _p(out["dphi"]),
+                                _p(out["db_pre"]), _p(out["db_post"]), _p(out["db_res"]),
+                                _p(out["dalpha"]), int(nthreads))
+    out["db_res"] = out["db_res"].reshape(n, n)
     return out
 
 

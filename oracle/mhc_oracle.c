@@ -151,3 +151,208 @@ void oracle_mhc_post(const double* X, const double* F_out, const double* H,
             }
     }
 }
+
+/* The normalised projection h = x_hat . phi of every token (the first two steps of the
+ * pre stage, equations rmsnorm and the projection of the "DeepSeek-V4/mhc" page).
+ * h [T, m]. */
+void oracle_mhc_projection(const double* X, const double* phi, long T, int n, int d,
+                           double eps, double* h, int nthreads)
+{
+    const int nd = n * d;
+    const int m = n * n + 2 * n;
+    if (nthreads <= 0) nthreads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (long t = 0; t < T; ++t) {
+        const double* Xt = X + t * (long)nd;
+        double* ht = h + t * (long)m;
+        double ss = 0.0;
+        for (int k = 0; k < nd; ++k) ss += Xt[k] * Xt[k];
+        const double r = sqrt(ss / (double)nd + eps);
+        for (int j = 0; j < m; ++j) ht[j] = 0.0;
+        for (int k = 0; k < nd; ++k)
+            for (int j = 0; j < m; ++j) ht[j] += (Xt[k] / r) * phi[(long)k * m + j];
+    }
+}
+
+/* Reverse mode through one token of pre + post (the chain rule applied to the forward
+ * steps above, last step first).  Accumulates into the per-thread parameter gradients
+ * gphi [nd*m], gb [m] (ordered [pre | res | post]) and ga [3] (pre, post, res: the order
+ * of the alpha arguments).
+ * work: [nd (x_hat) + nd (dx_hat) + m (h) + m (dl) + n*n*(2*t_max+1) (iterates) + 2*n*n]. */
+static void backward_one_token(const double* Xt, const double* Ft, const double* phi,
+                               const double* b_pre, const double* b_post, const double* b_res,
+                               double alpha_pre, double alpha_post, double alpha_res,
+                               int n, int d, double eps, int t_max,
+                               const double* dYt, const double* dxt,
+                               double* dXt, double* dFt, double* gphi, double* gb, double* ga,
+                               double* work)
+{
+    const int nd = n * d, nn = n * n, m = nn + 2 * n;
+    double* xhat = work;
+    double* dxhat = xhat + nd;
+    double* h = dxhat + nd;
+    double* dl = h + m;                   /* [dl_pre | dl_res | dl_post] */
+    double* it = dl + m;                  /* iterates M^(0..2 t_max), each n*n */
+    double* gM = it + nn * (2 * t_max + 1);
+    double* gA = gM + nn;
+
+    /* ---- forward, keeping what the reverse sweep needs */
+    double ss = 0.0;
+    for (int k = 0; k < nd; ++k) ss += Xt[k] * Xt[k];
+    const double r = sqrt(ss / (double)nd + eps);
+    for (int k = 0; k < nd; ++k) xhat[k] = Xt[k] / r;
+    for (int j = 0; j < m; ++j) h[j] = 0.0;
+    for (int k = 0; k < nd; ++k)
+        for (int j = 0; j < m; ++j) h[j] += xhat[k] * phi[(long)k * m + j];
+    double Hpre[8], Hpost[8];
+    for (int i = 0; i < n; ++i) Hpre[i] = sigmoid(alpha_pre * h[i] + b_pre[i]);
+    for (int i = 0; i < n; ++i) Hpost[i] = 2.0 * sigmoid(alpha_post * h[n + nn + i] + b_post[i]);
+    for (int q = 0; q < nn; ++q) it[q] = exp(alpha_res * h[n + q] + b_res[q]);
+    for (int s = 0; s < t_max; ++s) {
+        const double* A = it + (2 * s) * nn;
+        double* B = it + (2 * s + 1) * nn;      /* after the column step */
+        double* C = it + (2 * s + 2) * nn;      /* after the row step    */
+        for (int j = 0; j < n; ++j) {
+            double cs = 0.0;
+            for (int i = 0; i < n; ++i) cs += A[i * n + j];
+            for (int i = 0; i < n; ++i) B[i * n + j] = A[i * n + j] / cs;
+        }
+        for (int i = 0; i < n; ++i) {
+            double rs = 0.0;
+            for (int j = 0; j < n; ++j) rs += B[i * n + j];
+            for (int j = 0; j < n; ++j) C[i * n + j] = B[i * n + j] / rs;
+        }
+    }
+    const double* Hres = it + (2 * t_max) * nn;
+
+    /* ---- post: X' = H_res X + H_post^T F */
+    for (int k = 0; k < nd; ++k) dXt[k] = 0.0;
+    for (int q = 0; q < nn; ++q) gM[q] = 0.0;
+    double dHpost[8], dHpre[8];
+    for (int i = 0; i < n; ++i) {
+        dHpost[i] = 0.0;
+        for (int c = 0; c < d; ++c) dHpost[i] += dYt[i * d + c] * Ft[c];
+        for (int j = 0; j < n; ++j)
+            for (int c = 0; c < d; ++c) gM[i * n + j] += dYt[i * d + c] * Xt[j * d + c];
+    }
+    for (int j = 0; j < n; ++j)
+        for (int c = 0; c < d; ++c)
+            for (int i = 0; i < n; ++i) dXt[j * d + c] += Hres[i * n + j] * dYt[i * d + c];
+    for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += Hpost[i] * dYt[i * d + c];
+        dFt[c] = acc;
+    }
+    /* ---- read map: x_in = H_pre X */
+    for (int i = 0; i < n; ++i) {
+        dHpre[i] = 0.0;
+        for (int c = 0; c < d; ++c) dHpre[i] += dxt[c] * Xt[i * d + c];
+        for (int c = 0; c < d; ++c) dXt[i * d + c] += Hpre[i] * dxt[c];
+    }
+    /* ---- gates: sigmoid' = s (1 - s); H_post = 2 s */
+    for (int i = 0; i < n; ++i) dl[i] = dHpre[i] * Hpre[i] * (1.0 - Hpre[i]);
+    for (int i = 0; i < n; ++i) {
+        const double s = 0.5 * Hpost[i];
+        dl[n + nn + i] = dHpost[i] * 2.0 * s * (1.0 - s);
+    }
+    /* ---- Sinkhorn, last half-step first.  B = A / (row or column sum):
+     *      dA = (dB - <dB, B> over that row or column) / sum */
+    for (int s = t_max - 1; s >= 0; --s) {
+        const double* A = it + (2 * s) * nn;
+        const double* B = it + (2 * s + 1) * nn;
+        const double* C = it + (2 * s + 2) * nn;
+        for (int i = 0; i < n; ++i) {            /* row step: C = B / rowsum(B) */
+            double rs = 0.0, dot = 0.0;
+            for (int j = 0; j < n; ++j) { rs += B[i * n + j]; dot += gM[i * n + j] * C[i * n + j]; }
+            for (int j = 0; j < n; ++j) gA[i * n + j] = (gM[i * n + j] - dot) / rs;
+        }
+        for (int j = 0; j < n; ++j) {            /* column step: B = A / colsum(A) */
+            double cs = 0.0, dot = 0.0;
+            for (int i = 0; i < n; ++i) { cs += A[i * n + j]; dot += gA[i * n + j] * B[i * n + j]; }
+            for (int i = 0; i < n; ++i) gM[i * n + j] = (gA[i * n + j] - dot) / cs;
+        }
+    }
+    for (int q = 0; q < nn; ++q) dl[n + q] = gM[q] * it[q];      /* M0 = exp(l_res) */
+    /* ---- logits l = alpha h + b */
+    for (int j = 0; j < m; ++j) gb[j] += dl[j];
+    double dh[8 * 8 + 16];
+    for (int i = 0; i < n; ++i) { ga[0] += dl[i] * h[i]; dh[i] = alpha_pre * dl[i]; }
+    for (int q = 0; q < nn; ++q) { ga[2] += dl[n + q] * h[n + q]; dh[n + q] = alpha_res * dl[n + q]; }
+    for (int i = 0; i < n; ++i) {
+        ga[1] += dl[n + nn + i] * h[n + nn + i];
+        dh[n + nn + i] = alpha_post * dl[n + nn + i];
+    }
+    /* ---- projection h = x_hat phi */
+    for (int k = 0; k < nd; ++k) {
+        double acc = 0.0;
+        for (int j = 0; j < m; ++j) {
+            gphi[(long)k * m + j] += xhat[k] * dh[j];
+            acc += phi[(long)k * m + j] * dh[j];
+        }
+        dxhat[k] = acc;
+    }
+    /* ---- RMSNorm x_hat = v / r, r = sqrt(sum v^2 / nd + eps) */
+    double dot = 0.0;
+    for (int k = 0; k < nd; ++k) dot += dxhat[k] * Xt[k];
+    for (int k = 0; k < nd; ++k)
+        dXt[k] += dxhat[k] / r - Xt[k] * dot / ((double)nd * r * r * r);
+}
+
+void oracle_mhc_backward(const double* X, const double* F_out, const double* phi,
+                         const double* b_pre, const double* b_post, const double* b_res,
+                         double alpha_pre, double alpha_post, double alpha_res,
+                         long T, int n, int d, double eps, int t_max,
+                         const double* dX_out, const double* dx_in,
+                         double* dX, double* dF_out, double* dphi,
+                         double* db_pre, double* db_post, double* db_res, double* dalpha,
+                         int nthreads)
+{
+    const int nd = n * d, nn = n * n, m = nn + 2 * n;
+    if (nthreads <= 0) nthreads = 1;
+    const size_t wlen = (size_t)(2 * nd + 2 * m + nn * (2 * t_max + 1) + 2 * nn);
+    const size_t plen = (size_t)nd * m + m + 3;          /* per-thread parameter sums */
+    double* part = (double*)calloc((size_t)nthreads * plen, sizeof(double));
+#ifdef _OPENMP
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        tid = omp_get_thread_num();
+#endif
+        double* work = (double*)malloc(sizeof(double) * wlen);
+        double* gphi = part + (size_t)tid * plen;
+        double* gb = gphi + (size_t)nd * m;
+        double* ga = gb + m;
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
+        for (long t = 0; t < T; ++t)
+            backward_one_token(X + t * (long)nd, F_out + t * (long)d, phi, b_pre, b_post, b_res,
+                               alpha_pre, alpha_post, alpha_res, n, d, eps, t_max,
+                               dX_out + t * (long)nd, dx_in + t * (long)d,
+                               dX + t * (long)nd, dF_out + t * (long)d, gphi, gb, ga, work);
+        free(work);
+    }
+    /* thread partials summed in thread order */
+    for (size_t q = 0; q < (size_t)nd * m; ++q) {
+        double s = 0.0;
+        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + q];
+        dphi[q] = s;
+    }
+    for (int j = 0; j < m; ++j) {
+        double s = 0.0;
+        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + (size_t)nd * m + j];
+        if (j < n) db_pre[j] = s;
+        else if (j < n + nn) db_res[j - n] = s;
+        else db_post[j - n - nn] = s;
+    }
+    for (int a = 0; a < 3; ++a) {
+        double s = 0.0;
+        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + (size_t)nd * m + m + a];
+        dalpha[a] = s;
+    }
+    free(part);
+}

@@ -55,6 +55,27 @@ void oracle_mhc_pre(const double* X, const double* phi,
 void oracle_mhc_post(const double* X, const double* F_out, const double* H,
                      long T, int n, int d, double* X_out, int nthreads);
 
+/* The normalised projection h = RMSNorm(vec X_t) . phi of every token: h [T, m]. */
+void oracle_mhc_projection(const double* X, const double* phi, long T, int n, int d,
+                           double eps, double* h, int nthreads);
+
+/* Reverse mode of pre + post for the loss L = <dX_out, X'> + <dx_in, x_in>, i.e. the
+ * gradients of every input given the upstream gradients dX_out [T, n, d] (of X') and
+ * dx_in [T, d] (of x_in).  The chain rule applied to the forward's steps in reverse
+ * order; the Sinkhorn rounds are recomputed from the logits and their iterates kept in
+ * scratch.  Outputs: dX [T, n, d] (through the projection, RMSNorm, the read map and the
+ * merge), dF_out [T, d], dphi [n*d, m], db_pre [n], db_post [n], db_res [n*n] and
+ * dalpha [3] = (pre, post, res) -- the order of the alpha arguments -- the parameter
+ * gradients summed over all T tokens. */
+void oracle_mhc_backward(const double* X, const double* F_out, const double* phi,
+                         const double* b_pre, const double* b_post, const double* b_res,
+                         double alpha_pre, double alpha_post, double alpha_res,
+                         long T, int n, int d, double eps, int t_max,
+                         const double* dX_out, const double* dx_in,
+                         double* dX, double* dF_out, double* dphi,
+                         double* db_pre, double* db_post, double* db_res, double* dalpha,
+                         int nthreads);
+
 /* Number of OpenMP threads a parallel region with the given request uses. */
 int oracle_threads_used(int nthreads);
 
