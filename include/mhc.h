@@ -50,6 +50,7 @@
 #ifndef MHC_H
 #define MHC_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -67,7 +68,8 @@ typedef enum {
     MHC_ERR_DTYPE = 4,         /* dt is not an mhc_dtype value                       */
     MHC_ERR_UNSUPPORTED = 5,   /* the requested kernel path cannot run this problem  */
     MHC_ERR_CUDA = 6,          /* a CUDA call or launch failed                       */
-    MHC_ERR_ALIAS = 7          /* an output overlaps an input or another output      */
+    MHC_ERR_ALIAS = 7,         /* an output overlaps an input or another output      */
+    MHC_ERR_WORKSPACE = 8      /* workspace smaller than mhc_backward_workspace_bytes */
 } mhc_status;
 
 typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
@@ -129,6 +131,54 @@ mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt);
  */
 mhc_status mhc_post(const void* X, const void* F_out, const float* H, int64_t T, int n, int d,
                     mhc_dtype dt, void* X_out, mhc_stream_t stream);
+
+/*
+ * mhc_pre_train -- mhc_pre for training: the same computation and outputs, plus the
+ * normalised projection of every token, which mhc_backward needs to re-form the logits:
+ *   h[t, :] = (vec X_t / r_t) . phi                 [T, m] fp32, written in place
+ * (the "DeepSeek-V4/mhc" page, equations rmsnorm and the projection; the logits of
+ * equations a/b/c-tilde are alpha * h + b).  h may not overlap any other argument.
+ */
+mhc_status mhc_pre_train(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                         const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                         int64_t T, int n, int d, float eps, int t_max, mhc_dtype dt,
+                         void* x_in, float* H, float* h, mhc_stream_t stream);
+
+/*
+ * mhc_backward_workspace_bytes -- device workspace mhc_backward needs for (T, n, d); 0 for
+ * a shape it rejects.  Host-side, launches nothing.
+ */
+size_t mhc_backward_workspace_bytes(int64_t T, int n, int d);
+
+/*
+ * mhc_backward -- reverse mode of pre + post: the gradients of
+ *   L = <dX_out, X'> + <dx_in, x_in>
+ * with respect to X, F_out, phi, the biases and the three alphas, for the forward of
+ * mhc_pre / mhc_post above (the chain rule through each step of the "DeepSeek-V4/mhc"
+ * page's equations rmsnorm, a/b/c-tilde, gate, sinkhorn-init and sinkhorn, and the read
+ * map and merge of the slavadubrov.com Eq. 3, last step first).  The Sinkhorn rounds are
+ * recomputed from the pre-exp logits alpha_res * h_res + b_res; no iterate is stored.
+ * Inputs : X [T,n,d], F_out [T,d] (dt); phi [n*d, m]; b_pre [n], b_post [n], b_res [n*n];
+ *          alpha_*, eps, t_max as given to the forward; H [T,m] and h [T,m] as written by
+ *          mhc_pre_train; dX_out [T,n,d] (gradient of X') and dx_in [T,d] (gradient of
+ *          x_in), dt.
+ * Outputs: dX [T,n,d] and dF_out [T,d] (dt); dphi [n*d, m], db_pre [n], db_post [n],
+ *          db_res [n*n] and dalpha [3] = (pre, post, res), fp32, summed over all T tokens
+ *          in a fixed order (repeated calls give bitwise equal results).  For T == 0 the
+ *          parameter gradients are set to zero.
+ * workspace: device memory of at least mhc_backward_workspace_bytes(T, n, d) bytes,
+ *          256-byte aligned, owned by the caller, overwritten (else MHC_ERR_WORKSPACE).
+ * Limits : n <= 4 (MHC_ERR_UNSUPPORTED above); X, F_out, dX_out, dx_in, dX and dF_out
+ *          16-byte aligned with d * sizeof(element) a multiple of 16 (else MHC_ERR_ALIGN).
+ *          No output may overlap an input or another output (MHC_ERR_ALIAS).
+ */
+mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, const float* b_pre,
+                        const float* b_post, const float* b_res, float alpha_pre, float alpha_post,
+                        float alpha_res, const float* H, const float* h, int64_t T, int n, int d,
+                        float eps, int t_max, mhc_dtype dt, const void* dX_out, const void* dx_in,
+                        void* dX, void* dF_out, float* dphi, float* db_pre, float* db_post,
+                        float* db_res, float* dalpha, void* workspace, size_t workspace_bytes,
+                        mhc_stream_t stream);
 
 /*
  * mhc_device_status -- read and clear the device-side status word of the tensor-core

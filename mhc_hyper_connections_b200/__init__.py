@@ -8,6 +8,10 @@ CPU fallback -- if the library is missing the calls raise.
     mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
             x_in, H)                -> writes x_in [T, d] and H [T, n*n+2n]
     mhc_post(X, F_out, H, X_out)    -> writes X_out [T, n, d]
+    mhc_pre_train(..., x_in, H, h)  -> mhc_pre plus the normalised projection h [T, m]
+    mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+                 eps, t_max, H, h, dX_out, dx_in, dX, dF_out, dphi, db_pre, db_post,
+                 db_res, dalpha, workspace)  -> the gradients of <dX_out, X'> + <dx_in, x_in>
 
 Tensors are torch CUDA tensors (contiguous; X/F_out/x_in/X_out bf16 or fp32, phi, biases
 and H fp32).  Calls are asynchronous on the current torch stream unless ``stream`` (a
@@ -19,7 +23,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_post", "mhc_pre_path_for", "mhc_device_status",
+__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_post", "mhc_backward",
+           "mhc_backward_workspace_bytes", "mhc_pre_path_for", "mhc_device_status",
            "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
@@ -30,11 +35,13 @@ _LIB_PATH = os.path.join(_HERE, "libmhc_b200.so")
 MHC_F32, MHC_BF16 = 0, 1
 PRE_AUTO, PRE_GENERIC, PRE_CLUSTER_TC = 0, 1, 2
 _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN",
-           4: "MHC_ERR_DTYPE", 5: "MHC_ERR_UNSUPPORTED", 6: "MHC_ERR_CUDA", 7: "MHC_ERR_ALIAS"}
+           4: "MHC_ERR_DTYPE", 5: "MHC_ERR_UNSUPPORTED", 6: "MHC_ERR_CUDA", 7: "MHC_ERR_ALIAS",
+           8: "MHC_ERR_WORKSPACE"}
 
 # Every function include/mhc.h declares.
-EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_path_for", "mhc_post",
-                    "mhc_status_string", "mhc_last_error", "mhc_device_status")
+EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
+                    "mhc_backward_workspace_bytes", "mhc_backward", "mhc_status_string",
+                    "mhc_last_error", "mhc_device_status")
 
 _lock = threading.Lock()
 _lib = None
@@ -68,6 +75,13 @@ def load_library():
         lib.mhc_pre.restype = ci
         lib.mhc_pre_with_path.argtypes = pre_args + [ci]
         lib.mhc_pre_with_path.restype = ci
+        lib.mhc_pre_train.argtypes = pre_args[:-1] + [fp, vp]
+        lib.mhc_pre_train.restype = ci
+        lib.mhc_backward_workspace_bytes.argtypes = [i64, ci, ci]
+        lib.mhc_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.mhc_backward.argtypes = ([vp, vp, fp, fp, fp, fp, cf, cf, cf, fp, fp, i64, ci, ci, cf, ci, ci,
+                                      vp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ctypes.c_size_t, vp])
+        lib.mhc_backward.restype = ci
         lib.mhc_pre_path_for.argtypes = [i64, ci, ci, ci]
         lib.mhc_pre_path_for.restype = ci
         lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
@@ -179,6 +193,65 @@ def mhc_post(X, F_out, H, X_out, stream=None):
     with torch.cuda.device(dev):
         st = lib.mhc_post(px, pf, ph, T, n, d, _dt(X), po, _stream(stream, dev))
     _check(st, "mhc_post")
+
+
+def mhc_pre_train(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
+                  x_in, H, h, stream=None):
+    """mhc_pre plus the normalised projection h [T, n*n+2n] fp32 that mhc_backward needs."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    f32 = torch.float32
+    m = n * n + 2 * n
+    ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
+                b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
+                b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
+                H=_ptr(H, "H", f32, dev), h=_ptr(h, "h", f32, dev))
+    if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m) \
+            or tuple(h.shape) != (T, m):
+        raise ValueError("mhc_pre_train: shapes must be phi [n*d, m], x_in [T, d], H and h [T, m]")
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_pre_train(ptrs["X"], ptrs["phi"], ptrs["b_pre"], ptrs["b_post"], ptrs["b_res"],
+                               float(alpha_pre), float(alpha_post), float(alpha_res), T, n, d,
+                               float(eps), int(t_max), _dt(X), ptrs["x_in"], ptrs["H"], ptrs["h"],
+                               _stream(stream, dev))
+    _check(st, "mhc_pre_train")
+
+
+def mhc_backward_workspace_bytes(T: int, n: int, d: int) -> int:
+    """Bytes of device workspace mhc_backward needs (0 for a shape it rejects)."""
+    return int(load_library().mhc_backward_workspace_bytes(int(T), int(n), int(d)))
+
+
+def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
+                 H, h, dX_out, dx_in, dX, dF_out, dphi, db_pre, db_post, db_res, dalpha, workspace,
+                 stream=None):
+    """Gradients of <dX_out, X'> + <dx_in, x_in> (see include/mhc.h), written in place:
+    dX [T,n,d], dF_out [T,d] in X's dtype; dphi [n*d, m], db_pre [n], db_post [n],
+    db_res [n, n], dalpha [3] = (pre, post, res) fp32.  workspace: a CUDA tensor of at least
+    mhc_backward_workspace_bytes(T, n, d) bytes."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    f32 = torch.float32
+    dt = X.dtype
+    p = {k: _ptr(v, k, dt, dev) for k, v in dict(X=X, F_out=F_out, dX_out=dX_out, dx_in=dx_in,
+                                                  dX=dX, dF_out=dF_out).items()}
+    q = {k: _ptr(v, k, f32, dev) for k, v in dict(phi=phi, b_pre=b_pre, b_post=b_post, b_res=b_res,
+                                                   H=H, h=h, dphi=dphi, db_pre=db_pre,
+                                                   db_post=db_post, db_res=db_res,
+                                                   dalpha=dalpha).items()}
+    ws = _ptr(workspace, "workspace", device=dev)
+    nbytes = workspace.numel() * workspace.element_size()
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_backward(p["X"], p["F_out"], q["phi"], q["b_pre"], q["b_post"], q["b_res"],
+                              float(alpha_pre), float(alpha_post), float(alpha_res), q["H"], q["h"],
+                              T, n, d, float(eps), int(t_max), _dt(X), p["dX_out"], p["dx_in"],
+                              p["dX"], p["dF_out"], q["dphi"], q["db_pre"], q["db_post"],
+                              q["db_res"], q["dalpha"], ws, nbytes, _stream(stream, dev))
+    _check(st, "mhc_backward")
 
 
 def mhc_device_status() -> int:

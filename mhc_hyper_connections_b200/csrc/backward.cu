@@ -1,0 +1,409 @@
+// backward.cu -- reverse mode of the mHC layer (pre + post) for T tokens.
+//
+// It differentiates L = <dX_out, X'> + <dx_in, x_in> through the forward of include/mhc.h
+// ("DeepSeek-V4/mhc": equations rmsnorm, a/b/c-tilde, gate, sinkhorn-init, sinkhorn; the
+// slavadubrov.com Eq. 3 read map and merge), the chain rule taken step by step backwards.
+// With h the normalised projection the training forward saves, g = alpha * dl the
+// gradient of h, r the token's RMS and K = n*d:
+//
+//   post   dX += H_res^T dX_out, dF_out = H_post^T dX_out,
+//          dH_res[i][j] = <dX_out_i, X_j>, dH_post[i] = <dX_out_i, F_out>
+//   read   dX += H_pre dx_in, dH_pre[i] = <dx_in, X_i>
+//   gates  dl_pre = dH_pre H_pre (1 - H_pre), dl_post = dH_post H_post (1 - H_post / 2)
+//   SK     dl_res through the Sinkhorn rounds, recomputed from l_res = alpha_res h_res + b_res
+//   proj   dphi += (X_t / r) g^T,   dX_t += phi g / r - X_t (g . h) / (K r^2)
+//
+// The last term is the RMSNorm backward: sum_k (phi g)_k X_k = r (g . h), so no second
+// pass over the channels is needed.
+//
+// Kernels, in launch order:
+//   K1 bwd_reduce   warp per token: the sums over channels (sum X^2, dH_pre, dH_res,
+//                   dH_post) into a workspace row, and dF_out
+//   K2 bwd_token    thread per token: gates, Sinkhorn backward (O(t_max^2) recomputed
+//                   half-steps, nothing stored), G = g / r and beta = (g . h) / (K r^2)
+//   K3 bwd_dx_dphi  CTA per (channel slice, token group): dX, and the group's partial dphi
+//                   (each thread keeps one phi row and one dphi row in registers)
+//   K4 reductions   dphi over the groups, db and dalpha over the tokens, all in a fixed
+//                   order: repeated runs give bitwise equal results
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace mhc {
+namespace {
+
+constexpr int RED_THREADS = 256;
+constexpr int TOK_THREADS = 128;
+constexpr int DX_THREADS = 256;
+constexpr int TB = 32;               // tokens staged per batch in K3
+constexpr int SUM_THREADS = 256;
+
+__host__ __device__ constexpr int red_len(int n) { return 1 + n + n * n + n; }
+
+// ---------------------------------------------------------------- K1
+template <int N, typename T>
+__global__ void __launch_bounds__(RED_THREADS)
+bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __restrict__ dY,
+                  const T* __restrict__ dx, const float* __restrict__ H, int64_t Tn, int d,
+                  float* __restrict__ R, T* __restrict__ dF) {
+    constexpr int M = N * N + 2 * N, NR = red_len(N), V = Vec16<T>::VEC;
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int nchunk = d / V;
+    for (int64_t t = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < Tn; t += nwarps) {
+        float hpost[N];
+#pragma unroll
+        for (int i = 0; i < N; ++i) hpost[i] = __ldg(H + t * M + N + N * N + i);
+        float acc[NR];
+#pragma unroll
+        for (int q = 0; q < NR; ++q) acc[q] = 0.f;
+        for (int q = lane; q < nchunk; q += 32) {
+            float fx[N][V], fd[V], ff[V], df[V];
+#pragma unroll
+            for (int i = 0; i < N; ++i) Vec16<T>::unpack(ld_stream_v4(X + (t * N + i) * d + q * V), fx[i]);
+            Vec16<T>::unpack(ld_stream_v4(dx + t * d + q * V), fd);
+            Vec16<T>::unpack(ld_stream_v4(F + t * d + q * V), ff);
+#pragma unroll
+            for (int e = 0; e < V; ++e) df[e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    acc[0] = fmaf(fx[i][e], fx[i][e], acc[0]);
+                    acc[1 + i] = fmaf(fd[e], fx[i][e], acc[1 + i]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                float fy[V];
+                Vec16<T>::unpack(ld_stream_v4(dY + (t * N + i) * d + q * V), fy);
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    acc[1 + N + N * N + i] = fmaf(fy[e], ff[e], acc[1 + N + N * N + i]);
+                    df[e] = fmaf(hpost[i], fy[e], df[e]);
+#pragma unroll
+                    for (int j = 0; j < N; ++j)
+                        acc[1 + N + i * N + j] = fmaf(fy[e], fx[j][e], acc[1 + N + i * N + j]);
+                }
+            }
+            st_v4(dF + t * d + q * V, Vec16<T>::pack(df));
+        }
+#pragma unroll
+        for (int q = 0; q < NR; ++q) {
+            float v = acc[q];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            acc[q] = v;
+        }
+#pragma unroll
+        for (int q = 0; q < NR; ++q)
+            if (lane == (q & 31)) R[t * NR + q] = acc[q];
+    }
+}
+
+// ---------------------------------------------------------------- K2
+// Column then row normalisation of A (one Sinkhorn round); cs, rs receive the sums.
+template <int N>
+__device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], float (&C)[N][N],
+                                         float (&cs)[N], float (&rs)[N]) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < N; ++i) s += A[i][j];
+        cs[j] = s;
+#pragma unroll
+        for (int i = 0; i < N; ++i) B[i][j] = A[i][j] / s;
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) s += B[i][j];
+        rs[i] = s;
+#pragma unroll
+        for (int j = 0; j < N; ++j) C[i][j] = B[i][j] / s;
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(TOK_THREADS)
+bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const float* __restrict__ h,
+                 const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
+                 int64_t Tn, int K, float eps, int t_max, float* __restrict__ dl,
+                 float* __restrict__ G, float* __restrict__ beta) {
+    constexpr int M = N * N + 2 * N, NR = red_len(N);
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= Tn) return;
+    const float* Rt = R + t * NR;
+    float hh[M], out[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) hh[j] = h[t * M + j];
+    // gates
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const float hp = H[t * M + i];
+        out[i] = Rt[1 + i] * hp * (1.f - hp);
+        const float s = 0.5f * H[t * M + N + N * N + i];
+        out[N + N * N + i] = Rt[1 + N + N * N + i] * 2.f * s * (1.f - s);
+    }
+    // Sinkhorn: M0 = exp(l_res); the backward of round s needs its input A, recomputed
+    float M0[N][N], gM[N][N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            M0[i][j] = expf(a_res * hh[N + i * N + j] + b_res[i * N + j]);
+            gM[i][j] = Rt[1 + N + i * N + j];
+        }
+    for (int s = t_max - 1; s >= 0; --s) {
+        float A[N][N], B[N][N], C[N][N], cs[N], rs[N];
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+#pragma unroll
+            for (int j = 0; j < N; ++j) A[i][j] = M0[i][j];
+        for (int u = 0; u < s; ++u) {
+            sk_round<N>(A, B, C, cs, rs);
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+#pragma unroll
+                for (int j = 0; j < N; ++j) A[i][j] = C[i][j];
+        }
+        sk_round<N>(A, B, C, cs, rs);
+        // row step C = B / rowsum(B)
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < N; ++j) dot = fmaf(gM[i][j], C[i][j], dot);
+#pragma unroll
+            for (int j = 0; j < N; ++j) gM[i][j] = (gM[i][j] - dot) / rs[i];
+        }
+        // column step B = A / colsum(A)
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            float dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < N; ++i) dot = fmaf(gM[i][j], B[i][j], dot);
+#pragma unroll
+            for (int i = 0; i < N; ++i) gM[i][j] = (gM[i][j] - dot) / cs[j];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int j = 0; j < N; ++j) out[N + i * N + j] = gM[i][j] * M0[i][j];
+    // g = alpha * dl; G = g / r; beta = (g . h) / (K r^2)
+    const float inv_r = 1.0f / sqrtf(Rt[0] / (float)K + eps);
+    float gh = 0.f;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+        const float a = j < N ? a_pre : (j < N + N * N ? a_res : a_post);
+        const float g = a * out[j];
+        gh = fmaf(g, hh[j], gh);
+        dl[t * M + j] = out[j];
+        G[t * M + j] = g * inv_r;
+    }
+    beta[t] = gh * inv_r * inv_r / (float)K;
+}
+
+// ---------------------------------------------------------------- K3
+// Channel slice [c0, c0 + CS) of all N streams: thread (i, c) owns phi row i*d + c.
+template <int N, typename T>
+__global__ void __launch_bounds__(DX_THREADS)
+bwd_dx_dphi_kernel(const T* __restrict__ X, const T* __restrict__ dY, const T* __restrict__ dx,
+                   const float* __restrict__ phi, const float* __restrict__ H,
+                   const float* __restrict__ G, const float* __restrict__ beta, int64_t Tn, int d,
+                   int tpg, T* __restrict__ dX, float* __restrict__ part) {
+    constexpr int M = N * N + 2 * N;
+    constexpr int CS = DX_THREADS / N >= 256 ? 256 : (DX_THREADS / N >= 128 ? 128 : 64);
+    __shared__ float sG[TB][M], sH[TB][M], sB[TB];
+    const int i = threadIdx.x / CS;
+    const int c = blockIdx.x * CS + (threadIdx.x % CS);
+    const bool active = i < N && c < d;
+    const int64_t k = (int64_t)i * d + c;
+    const int K = N * d;
+    float prow[M], acc[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+        prow[j] = active ? __ldg(phi + k * M + j) : 0.f;
+        acc[j] = 0.f;
+    }
+    const int64_t t_lo = (int64_t)blockIdx.y * tpg;
+    const int64_t t_hi = t_lo + tpg < Tn ? t_lo + tpg : Tn;
+    for (int64_t tb = t_lo; tb < t_hi; tb += TB) {
+        const int nb = (int)(t_hi - tb < TB ? t_hi - tb : TB);
+        __syncthreads();
+        for (int e = threadIdx.x; e < nb * M; e += blockDim.x) {
+            const int u = e / M, j = e - u * M;
+            sG[u][j] = G[(tb + u) * M + j];
+            sH[u][j] = H[(tb + u) * M + j];
+        }
+        for (int u = threadIdx.x; u < nb; u += blockDim.x) sB[u] = beta[tb + u];
+        __syncthreads();
+        if (!active) continue;
+        for (int u = 0; u < nb; ++u) {
+            const int64_t t = tb + u;
+            const float v = to_f32(X[t * K + k]);
+            float pg = 0.f;
+#pragma unroll
+            for (int j = 0; j < M; ++j) {
+                acc[j] = fmaf(v, sG[u][j], acc[j]);
+                pg = fmaf(prow[j], sG[u][j], pg);
+            }
+            float g = sH[u][i] * to_f32(dx[t * d + c]) + pg - sB[u] * v;
+#pragma unroll
+            for (int q = 0; q < N; ++q) g = fmaf(sH[u][N + q * N + i], to_f32(dY[t * K + (int64_t)q * d + c]), g);
+            store_elem(&dX[t * K + k], g);
+        }
+    }
+    if (active) {
+        float* p = part + ((int64_t)blockIdx.y * K + k) * M;
+#pragma unroll
+        for (int j = 0; j < M; ++j) p[j] = acc[j];
+    }
+}
+
+// ---------------------------------------------------------------- K4
+// dphi = sum over the token groups of the partials, in group order.
+__global__ void __launch_bounds__(SUM_THREADS)
+bwd_dphi_sum_kernel(const float* __restrict__ part, int64_t len, int groups, float* __restrict__ dphi) {
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < len;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int g = 0; g < groups; ++g) s += part[(int64_t)g * len + e];
+        dphi[e] = s;
+    }
+}
+
+// Column j (one CTA each): colsum[j] = sum_t dl[t][j] and colsum[M + j] = sum_t dl[t][j] h[t][j];
+// each thread sums a fixed strided set of tokens, then a fixed-order tree.
+__global__ void __launch_bounds__(SUM_THREADS)
+bwd_colsum_kernel(const float* __restrict__ dl, const float* __restrict__ h, int64_t Tn, int M,
+                  float* __restrict__ colsum) {
+    __shared__ float s0[SUM_THREADS], s1[SUM_THREADS];
+    const int j = blockIdx.x;
+    float a = 0.f, b = 0.f;
+    for (int64_t t = threadIdx.x; t < Tn; t += SUM_THREADS) {
+        const float v = dl[t * M + j];
+        a += v;
+        b = fmaf(v, h[t * M + j], b);
+    }
+    s0[threadIdx.x] = a;
+    s1[threadIdx.x] = b;
+    __syncthreads();
+    for (int w = SUM_THREADS / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) {
+            s0[threadIdx.x] += s0[threadIdx.x + w];
+            s1[threadIdx.x] += s1[threadIdx.x + w];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        colsum[j] = s0[0];
+        colsum[M + j] = s1[0];
+    }
+}
+
+// db from the column sums; dalpha = (pre, post, res) sums of the dl * h column sums.
+__global__ void bwd_bias_alpha_kernel(const float* __restrict__ colsum, int n, float* __restrict__ db_pre,
+                                      float* __restrict__ db_post, float* __restrict__ db_res,
+                                      float* __restrict__ dalpha) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const int nn = n * n, M = nn + 2 * n;
+    float ap = 0.f, ar = 0.f, aq = 0.f;
+    for (int j = 0; j < n; ++j) { db_pre[j] = colsum[j]; ap += colsum[M + j]; }
+    for (int q = 0; q < nn; ++q) { db_res[q] = colsum[n + q]; ar += colsum[M + n + q]; }
+    for (int j = 0; j < n; ++j) { db_post[j] = colsum[n + nn + j]; aq += colsum[M + n + nn + j]; }
+    dalpha[0] = ap;
+    dalpha[1] = aq;
+    dalpha[2] = ar;
+}
+
+int dx_slice(int n) { return DX_THREADS / n >= 256 ? 256 : (DX_THREADS / n >= 128 ? 128 : 64); }
+
+template <int N, typename T>
+cudaError_t launch_n(const BwdArgs& a, const BwdLayout& L) {
+    constexpr int M = N * N + 2 * N;
+    const int64_t Tn = a.T;
+    const int d = a.d, K = N * d;
+    const T* X = static_cast<const T*>(a.X);
+    const T* dY = static_cast<const T*>(a.dX_out);
+    const T* dxi = static_cast<const T*>(a.dx_in);
+    float* ws = static_cast<float*>(a.workspace);
+    float* R = ws + L.off_R;
+    float* dl = ws + L.off_dl;
+    float* G = ws + L.off_G;
+    float* beta = ws + L.off_beta;
+    float* part = ws + L.off_part;
+    float* colsum = ws + L.off_colsum;
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    {
+        int64_t blocks = (Tn * 32 + RED_THREADS - 1) / RED_THREADS;
+        const int64_t cap = (int64_t)di.sm_count * 8;
+        if (blocks > cap) blocks = cap;
+        bwd_reduce_kernel<N, T><<<(unsigned)blocks, RED_THREADS, 0, a.stream>>>(
+            X, static_cast<const T*>(a.F), dY, dxi, a.H, Tn, d, R, static_cast<T*>(a.dF_out));
+    }
+    bwd_token_kernel<N><<<(unsigned)((Tn + TOK_THREADS - 1) / TOK_THREADS), TOK_THREADS, 0, a.stream>>>(
+        R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res, Tn, K, a.eps, a.t_max, dl, G, beta);
+    {
+        const int cs = dx_slice(N);
+        dim3 grid((unsigned)((d + cs - 1) / cs), (unsigned)L.groups);
+        bwd_dx_dphi_kernel<N, T><<<grid, DX_THREADS, 0, a.stream>>>(
+            X, dY, dxi, a.phi, a.H, G, beta, Tn, d, L.tokens_per_group, static_cast<T*>(a.dX), part);
+    }
+    {
+        const int64_t len = (int64_t)K * M;
+        int64_t blocks = (len + SUM_THREADS - 1) / SUM_THREADS;
+        if (blocks > (int64_t)di.sm_count * 8) blocks = (int64_t)di.sm_count * 8;
+        bwd_dphi_sum_kernel<<<(unsigned)blocks, SUM_THREADS, 0, a.stream>>>(part, len, L.groups, a.dphi);
+    }
+    bwd_colsum_kernel<<<M, SUM_THREADS, 0, a.stream>>>(dl, a.h, Tn, M, colsum);
+    bwd_bias_alpha_kernel<<<1, 32, 0, a.stream>>>(colsum, N, a.db_pre, a.db_post, a.db_res, a.dalpha);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch(const BwdArgs& a, const BwdLayout& L) {
+    switch (a.n) {
+        case 1: return launch_n<1, T>(a, L);
+        case 2: return launch_n<2, T>(a, L);
+        case 3: return launch_n<3, T>(a, L);
+        case 4: return launch_n<4, T>(a, L);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+BwdLayout backward_layout(int64_t T, int n, int d) {
+    BwdLayout L{};
+    const int64_t m = (int64_t)n * n + 2 * n, K = (int64_t)n * d;
+    const int64_t slices = (d + dx_slice(n) - 1) / dx_slice(n);
+    // about 1024 CTAs in K3, each group at least 32 tokens
+    int64_t groups = (1024 + slices - 1) / slices;
+    const int64_t max_groups = (T + TB - 1) / TB;
+    if (groups > max_groups) groups = max_groups;
+    if (groups < 1) groups = 1;
+    L.groups = (int)groups;
+    L.tokens_per_group = (T + groups - 1) / groups;
+    auto up = [](int64_t x) { return (x + 63) / 64 * 64; };   // 256-byte aligned regions
+    int64_t off = 0;
+    L.off_R = off;      off += up(T * red_len(n));
+    L.off_dl = off;     off += up(T * m);
+    L.off_G = off;      off += up(T * m);
+    L.off_beta = off;   off += up(T);
+    L.off_part = off;   off += up(groups * K * m);
+    L.off_colsum = off; off += up(2 * m);
+    L.floats = off;
+    return L;
+}
+
+cudaError_t launch_backward(const BwdArgs& a) {
+    const BwdLayout L = backward_layout(a.T, a.n, a.d);
+    return a.dt == BF16 ? dispatch<__nv_bfloat16>(a, L) : dispatch<float>(a, L);
+}
+
+}  // namespace mhc

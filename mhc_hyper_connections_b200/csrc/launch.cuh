@@ -22,6 +22,7 @@ struct PreArgs {
     DType dt;
     void* x_in;
     float* H;
+    float* h_out = nullptr;      // optional [T, m]: the normalised projection, for the backward
     cudaStream_t stream;
 };
 
@@ -56,5 +57,41 @@ cudaError_t launch_pre_cluster_tc(const PreArgs& a);
 cudaError_t pre_cluster_tc_status(unsigned* out, bool clear);
 
 cudaError_t launch_post(const PostArgs& a);
+
+// Reverse mode of pre + post (backward.cu).
+struct BwdArgs {
+    const void* X;
+    const void* F;
+    const float* phi;
+    const float* b_res;
+    float a_pre, a_post, a_res;
+    const float* H;              // forward coefficients [T, m]
+    const float* h;              // saved normalised projection [T, m]
+    int64_t T;
+    int n, d;
+    float eps;
+    int t_max;
+    DType dt;
+    const void* dX_out;
+    const void* dx_in;
+    void* dX;
+    void* dF_out;
+    float* dphi;
+    float* db_pre;
+    float* db_post;
+    float* db_res;
+    float* dalpha;
+    void* workspace;
+    cudaStream_t stream;
+};
+
+// Workspace regions, in floats from the (256-byte aligned) workspace base.
+struct BwdLayout {
+    int64_t off_R, off_dl, off_G, off_beta, off_part, off_colsum, floats;
+    int groups;                  // token groups of the dX / dphi kernel
+    int64_t tokens_per_group;
+};
+BwdLayout backward_layout(int64_t T, int n, int d);
+cudaError_t launch_backward(const BwdArgs& a);
 
 }  // namespace mhc

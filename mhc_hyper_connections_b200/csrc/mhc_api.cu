@@ -119,19 +119,19 @@ mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
     return MHC_PRE_GENERIC;
 }
 
-mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre,
-                             const float* b_post, const float* b_res, float alpha_pre,
-                             float alpha_post, float alpha_res, int64_t T, int n, int d,
-                             float eps, int t_max, mhc_dtype dt, void* x_in, float* H,
-                             mhc_stream_t stream, mhc_pre_path path) {
+static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                           const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                           int64_t T, int n, int d, float eps, int t_max, mhc_dtype dt, void* x_in,
+                           float* H, float* h_out, mhc_stream_t stream, mhc_pre_path path) {
     mhc_status st = validate_pre(X, phi, b_pre, b_post, b_res, T, n, d, t_max, dt, x_in, H);
     if (st != MHC_OK) return st;
     if (path != MHC_PRE_AUTO && path != MHC_PRE_GENERIC && path != MHC_PRE_CLUSTER_TC)
         return MHC_ERR_UNSUPPORTED;
     if (T == 0) return MHC_OK;
     if (path == MHC_PRE_AUTO) path = mhc_pre_path_for(T, n, d, dt);
-    const PreArgs a = make_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T,
-                               n, d, eps, t_max, dt, x_in, H, stream);
+    PreArgs a = make_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T,
+                         n, d, eps, t_max, dt, x_in, H, stream);
+    a.h_out = h_out;
     cudaError_t e;
     if (path == MHC_PRE_CLUSTER_TC) {
         if (!pre_cluster_tc_shape_ok(T, n, d, a.dt) || !pre_cluster_tc_device_ok(n, d))
@@ -143,6 +143,102 @@ mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre
         e = launch_pre_generic(a);
         if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (generic kernel)");
     }
+    return MHC_OK;
+}
+
+mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre,
+                             const float* b_post, const float* b_res, float alpha_pre,
+                             float alpha_post, float alpha_res, int64_t T, int n, int d,
+                             float eps, int t_max, mhc_dtype dt, void* x_in, float* H,
+                             mhc_stream_t stream, mhc_pre_path path) {
+    return pre_impl(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T, n, d, eps,
+                    t_max, dt, x_in, H, nullptr, stream, path);
+}
+
+mhc_status mhc_pre_train(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                         const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                         int64_t T, int n, int d, float eps, int t_max, mhc_dtype dt, void* x_in,
+                         float* H, float* h, mhc_stream_t stream) {
+    mhc_status st = check_shape(T, n, d, dt);
+    if (st != MHC_OK) return st;
+    if (T > 0) {
+        if (!h) return MHC_ERR_NULL;
+        if (!aligned(h, 4)) return MHC_ERR_ALIGN;
+        const int m = n * n + 2 * n;
+        const size_t es = elem_size(dt), nh = (size_t)T * m * 4;
+        const void* other[7] = {X, phi, b_pre, b_post, b_res, x_in, H};
+        const size_t nother[7] = {(size_t)T * n * d * es, (size_t)n * d * m * 4, (size_t)n * 4,
+                                  (size_t)n * 4, (size_t)n * n * 4, (size_t)T * d * es, nh};
+        for (int i = 0; i < 7; ++i)
+            if (overlaps(h, nh, other[i], nother[i])) return MHC_ERR_ALIAS;
+    }
+    return pre_impl(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T, n, d, eps,
+                    t_max, dt, x_in, H, h, stream, MHC_PRE_AUTO);
+}
+
+size_t mhc_backward_workspace_bytes(int64_t T, int n, int d) {
+    if (check_shape(T, n, d, MHC_F32) != MHC_OK || n > 4) return 0;
+    return (size_t)backward_layout(T, n, d).floats * 4;
+}
+
+mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, const float* b_pre,
+                        const float* b_post, const float* b_res, float alpha_pre, float alpha_post,
+                        float alpha_res, const float* H, const float* h, int64_t T, int n, int d,
+                        float eps, int t_max, mhc_dtype dt, const void* dX_out, const void* dx_in,
+                        void* dX, void* dF_out, float* dphi, float* db_pre, float* db_post,
+                        float* db_res, float* dalpha, void* workspace, size_t workspace_bytes,
+                        mhc_stream_t stream) {
+    mhc_status st = check_shape(T, n, d, dt);
+    if (st != MHC_OK) return st;
+    if (t_max < 0 || t_max > 1000) return MHC_ERR_SHAPE;
+    if (n > 4) return MHC_ERR_UNSUPPORTED;
+    if (!phi || !b_pre || !b_post || !b_res || !dphi || !db_pre || !db_post || !db_res || !dalpha)
+        return MHC_ERR_NULL;
+    const int m = n * n + 2 * n;
+    const size_t es = elem_size(dt);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t nphi = (size_t)n * d * m * 4;
+    if (T == 0) {   // no tokens: every parameter gradient is zero
+        cudaError_t e = cudaMemsetAsync(dphi, 0, nphi, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(db_pre, 0, (size_t)n * 4, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(db_post, 0, (size_t)n * 4, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(db_res, 0, (size_t)n * n * 4, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dalpha, 0, 3 * 4, s);
+        return e == cudaSuccess ? MHC_OK : cuda_fail(e, "mhc_backward");
+    }
+    if (!X || !F_out || !H || !h || !dX_out || !dx_in || !dX || !dF_out || !workspace) return MHC_ERR_NULL;
+    const void* vec[6] = {X, F_out, dX_out, dx_in, dX, dF_out};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned(vec[i], 16)) return MHC_ERR_ALIGN;
+    if ((size_t)d * es % 16 != 0) return MHC_ERR_ALIGN;
+    const float* f4[9] = {phi, b_pre, b_post, b_res, H, h, dphi, db_pre, db_post};
+    for (int i = 0; i < 9; ++i)
+        if (!aligned(f4[i], 4)) return MHC_ERR_ALIGN;
+    if (!aligned(db_res, 4) || !aligned(dalpha, 4) || !aligned(workspace, 256)) return MHC_ERR_ALIGN;
+    const size_t need = mhc_backward_workspace_bytes(T, n, d);
+    if (workspace_bytes < need) return MHC_ERR_WORKSPACE;
+    const size_t nX = (size_t)T * n * d * es, nD = (size_t)T * d * es, nH = (size_t)T * m * 4;
+    const void* ins[10] = {X, F_out, phi, b_pre, b_post, b_res, H, h, dX_out, dx_in};
+    const size_t nins[10] = {nX, nD, nphi, (size_t)n * 4, (size_t)n * 4, (size_t)n * n * 4, nH, nH, nX, nD};
+    void* outs[8] = {dX, dF_out, dphi, db_pre, db_post, db_res, dalpha, workspace};
+    const size_t nouts[8] = {nX, nD, nphi, (size_t)n * 4, (size_t)n * 4, (size_t)n * n * 4, 12, need};
+    for (int o = 0; o < 8; ++o) {
+        for (int i = 0; i < 10; ++i)
+            if (overlaps(outs[o], nouts[o], ins[i], nins[i])) return MHC_ERR_ALIAS;
+        for (int p = o + 1; p < 8; ++p)
+            if (overlaps(outs[o], nouts[o], outs[p], nouts[p])) return MHC_ERR_ALIAS;
+    }
+    BwdArgs a;
+    a.X = X; a.F = F_out; a.phi = phi; a.b_res = b_res;
+    a.a_pre = alpha_pre; a.a_post = alpha_post; a.a_res = alpha_res;
+    a.H = H; a.h = h; a.T = T; a.n = n; a.d = d; a.eps = eps; a.t_max = t_max;
+    a.dt = dt == MHC_BF16 ? BF16 : F32;
+    a.dX_out = dX_out; a.dx_in = dx_in; a.dX = dX; a.dF_out = dF_out; a.dphi = dphi;
+    a.db_pre = db_pre; a.db_post = db_post; a.db_res = db_res; a.dalpha = dalpha;
+    a.workspace = workspace;
+    a.stream = s;
+    cudaError_t e = launch_backward(a);
+    if (e != cudaSuccess) return cuda_fail(e, "mhc_backward");
     return MHC_OK;
 }
 
@@ -188,6 +284,7 @@ const char* mhc_status_string(mhc_status s) {
         case MHC_ERR_UNSUPPORTED: return "the requested kernel path cannot run this problem";
         case MHC_ERR_CUDA: return "a CUDA call or launch failed (see mhc_last_error)";
         case MHC_ERR_ALIAS: return "an output overlaps an input or another output";
+        case MHC_ERR_WORKSPACE: return "the workspace is smaller than mhc_backward_workspace_bytes";
     }
     return "unknown status";
 }

@@ -129,7 +129,7 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
                       const float* __restrict__ b_pre, const float* __restrict__ b_post,
                       const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                       int T, int d, float eps, int t_max, __nv_bfloat16* __restrict__ x_in,
-                      float* __restrict__ H, int ncb, int nstage)
+                      float* __restrict__ H, float* __restrict__ h_out, int ncb, int nstage)
 {
     using C = Cfg<N>;
     constexpr int M = C::M;
@@ -318,6 +318,10 @@ pre_cluster_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* _
             }
             const float inv_r = 1.0f / sqrtf(ss * invK + eps);
             const float z = alpha * (h * inv_r) + bias;
+            if (h_out != nullptr && lane < M) {   // the normalised projection, for the backward
+                const int64_t tok = (int64_t)(cid + k * ncl) * NT + rank;
+                if (tok < T) h_out[tok * M + lane] = h * inv_r;
+            }
             const float hp = lane < N ? sigmoid_f32(z) : 0.f;
             float hv[4];
 #pragma unroll
@@ -665,7 +669,7 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p, int ncb) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, pre_cluster_tc_kernel<N>, map, a.phi, a.b_pre, a.b_post, a.b_res,
                               a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps, a.t_max,
-                              static_cast<__nv_bfloat16*>(a.x_in), a.H, ncb, p.nstage);
+                              static_cast<__nv_bfloat16*>(a.x_in), a.H, a.h_out, ncb, p.nstage);
 }
 
 }  // namespace tc

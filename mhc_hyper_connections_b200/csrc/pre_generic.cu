@@ -24,7 +24,7 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
                    const float* __restrict__ b_pre, const float* __restrict__ b_post,
                    const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                    int64_t Tn, int d, float eps, int t_max, T* __restrict__ x_in,
-                   float* __restrict__ H)
+                   float* __restrict__ H, float* __restrict__ h_out)
 {
     constexpr int M = N * N + 2 * N;
     constexpr int NO = (TT * M + THREADS - 1) / THREADS;   // projection outputs per thread
@@ -90,9 +90,14 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
         const int64_t tok = t0 + tid;
         const float r = sqrtf(ss_s[tid] / (float)K + eps);
         float out[M];
-        token_maps<N>(hs[tid], 1.0f / r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+        const float inv_r = 1.0f / r;
+        token_maps<N>(hs[tid], inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
 #pragma unroll
         for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
+        if (h_out != nullptr) {        // the normalised projection, as the logits use it
+#pragma unroll
+            for (int j = 0; j < M; ++j) h_out[tok * M + j] = hs[tid][j] * inv_r;
+        }
 #pragma unroll
         for (int i = 0; i < N; ++i) hpre_s[tid][i] = out[i];
     }
@@ -115,7 +120,7 @@ cudaError_t launch_n(const PreArgs& a) {
     if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
     pre_generic_kernel<N, T><<<(unsigned)blocks, THREADS, 0, a.stream>>>(
         static_cast<const T*>(a.X), a.phi, a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post,
-        a.a_res, a.T, a.d, a.eps, a.t_max, static_cast<T*>(a.x_in), a.H);
+        a.a_res, a.T, a.d, a.eps, a.t_max, static_cast<T*>(a.x_in), a.H, a.h_out);
     return cudaGetLastError();
 }
 
