@@ -400,6 +400,130 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_backward(args, rank, world, local_rank):
+    """Forward + backward steps (mhc_pre_train, mhc_post, mhc_backward) on one batch: the
+    backward workload (T=16384, n=4, d=4096, bf16 with outlier channels, upstream gradients
+    dX_out and dx_in ~ N(0,1) in bf16).  Prints one JSON line."""
+    import numpy as np
+    import torch
+
+    import mhc_hyper_connections_b200 as mhc
+    from mhc_hyper_connections_b200 import dist as mdist
+    from mhc_hyper_connections_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    w = wl.make_config(args.config)
+    if args.tokens:
+        w = w.tokens(np.arange(min(args.tokens, w.T)))
+    T, n, d, m = w.T, w.n, w.d, w.m
+    es = 2 if w.dtype == "bf16" else 4
+    rng = np.random.default_rng(1000 + rank)
+    up = [rng.standard_normal(sh, dtype=np.float32) for sh in ((T, n, d), (T, d))]
+    if w.dtype == "bf16":
+        up = [wl.bf16_round_bits(a) for a in up]
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    X, F, dY, dxi = to_dev(w.X), to_dev(w.F_out), to_dev(up[0]), to_dev(up[1])
+    phi, b_pre, b_post, b_res = (to_dev(a) for a in (w.phi, w.b_pre, w.b_post, w.b_res))
+    x_in = torch.empty(T, d, dtype=X.dtype, device=dev)
+    H = torch.empty(T, m, device=dev)
+    h = torch.empty(T, m, device=dev)
+    Y = torch.empty_like(X)
+    dX, dF = torch.empty_like(X), torch.empty_like(F)
+    dphi = torch.empty(n * d, m, device=dev)
+    db_pre, db_post, db_res = (torch.empty(n, device=dev), torch.empty(n, device=dev),
+                               torch.empty(n, n, device=dev))
+    dalpha = torch.empty(3, device=dev)
+    ws = torch.empty(mhc.mhc_backward_workspace_bytes(T, n, d), dtype=torch.uint8, device=dev)
+    s = w.scalars()
+    sa = (s["alpha_pre"], s["alpha_post"], s["alpha_res"], s["eps"], s["t_max"])
+
+    def fwd():
+        mhc.mhc_pre_train(X, phi, b_pre, b_post, b_res, *sa, x_in, H, h)
+
+    def post():
+        mhc.mhc_post(X, F, H, Y)
+
+    def bwd():
+        mhc.mhc_backward(X, F, phi, b_pre, b_post, b_res, *sa, H, h, dY, dxi, dX, dF, dphi,
+                         db_pre, db_post, db_res, dalpha, ws)
+
+    for _ in range(args.warmup):
+        fwd(); post(); bwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local_rank)
+    clk.start()
+    time.sleep(0.6)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record()
+    for k in range(K):
+        e = evs[k]
+        e[0].record(); fwd(); e[1].record(); post(); e[2].record(); bwd(); e[3].record()
+    end.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    time.sleep(0.3)
+    clk.stop()
+    ms_total = mdist.max_over_ranks(start.elapsed_time(end), device=dev)
+    st = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(3)]
+    value = mdist.job_throughput(T, K, ms_total, world)
+    peak, peak_src = _hbm_peak()
+    by_pre, by_post = bytes_per_token(n, d, es)
+    by_pre += 4 * m                                            # the saved projection h
+    # backward, dependency-minimal: read X, F_out, dX_out, dx_in, H, h; write dX, dF_out
+    by_bwd = (3 * n + 3) * d * es + 8 * m
+    bw_gbs = by_bwd * T / (st[2] / 1e3) / 1e9
+    step_bytes = (by_pre + by_post + by_bwd) * T
+    step_gbs = step_bytes / (ms_total / 1e3 / K) / 1e9       # per GPU: each processes T tokens
+    line = {
+        "metric": "mHC forward+backward tokens/s (pre_train + post + backward), n=4 d=4096 bf16",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": args.config + "+backward", "T": T, "n": n, "d": d,
+                   "upstream": "dX_out, dx_in ~ N(0,1), stored like X",
+                   "l2": "inputs larger than L2, no flush"},
+        "kernels": {"pre_train": {"ms": st[0], "bytes_per_launch": by_pre * T,
+                                  "gbs": by_pre * T / (st[0] / 1e3) / 1e9},
+                    "post": {"ms": st[1], "bytes_per_launch": by_post * T,
+                             "gbs": by_post * T / (st[1] / 1e3) / 1e9},
+                    "backward": {"ms": st[2], "bytes_per_launch": by_bwd * T, "gbs": bw_gbs,
+                                 "launches": 6,
+                                 "source": "mhc_hyper_connections_b200/csrc/backward.cu"}},
+        "roofline": {"kernel": "backward (6 launches)", "bound": "hbm", "achieved": bw_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": bw_gbs / peak, "traffic": None,
+                     "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": by_bwd * T},
+        "hbm": {"step_bytes_per_token": by_pre + by_post + by_bwd, "gbs_per_gpu": step_gbs,
+                "frac_of_measured": step_gbs / peak},
+        "clocks": clk.summary(t_wall0, t_wall1), "e2e": None, "cpu_baseline": None,
+        "gpu_launches": 8 * K,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def main():
     from mhc_hyper_connections_b200 import workloads as wl
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
@@ -417,6 +541,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--backward", action="store_true",
+                    help="time forward + backward steps (mhc_pre_train, mhc_post, mhc_backward)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -428,6 +554,8 @@ def main():
             ap.error("--gpus N > 1 needs one process per GPU (torchrun --nproc-per-node N)")
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.backward:
+        return run_backward(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 

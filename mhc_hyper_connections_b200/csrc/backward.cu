@@ -35,6 +35,7 @@ constexpr int RED_THREADS = 256;
 constexpr int TOK_THREADS = 128;
 constexpr int DX_THREADS = 256;
 constexpr int TB = 32;               // tokens staged per batch in K3
+constexpr int UN = 8;                // tokens whose loads K3 has in flight at once
 constexpr int SUM_THREADS = 256;
 
 __host__ __device__ constexpr int red_len(int n) { return 1 + n + n * n + n; }
@@ -101,7 +102,8 @@ bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __r
 }
 
 // ---------------------------------------------------------------- K2
-// Column then row normalisation of A (one Sinkhorn round); cs, rs receive the sums.
+// Column then row normalisation of A (one Sinkhorn round); cs, rs receive the reciprocals
+// of the column and row sums.
 template <int N>
 __device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], float (&C)[N][N],
                                          float (&cs)[N], float (&rs)[N]) {
@@ -110,18 +112,18 @@ __device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], flo
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < N; ++i) s += A[i][j];
-        cs[j] = s;
+        cs[j] = 1.0f / s;
 #pragma unroll
-        for (int i = 0; i < N; ++i) B[i][j] = A[i][j] / s;
+        for (int i = 0; i < N; ++i) B[i][j] = A[i][j] * cs[j];
     }
 #pragma unroll
     for (int i = 0; i < N; ++i) {
         float s = 0.f;
 #pragma unroll
         for (int j = 0; j < N; ++j) s += B[i][j];
-        rs[i] = s;
+        rs[i] = 1.0f / s;
 #pragma unroll
-        for (int j = 0; j < N; ++j) C[i][j] = B[i][j] / s;
+        for (int j = 0; j < N; ++j) C[i][j] = B[i][j] * rs[i];
     }
 }
 
@@ -176,7 +178,7 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
 #pragma unroll
             for (int j = 0; j < N; ++j) dot = fmaf(gM[i][j], C[i][j], dot);
 #pragma unroll
-            for (int j = 0; j < N; ++j) gM[i][j] = (gM[i][j] - dot) / rs[i];
+            for (int j = 0; j < N; ++j) gM[i][j] = (gM[i][j] - dot) * rs[i];
         }
         // column step B = A / colsum(A)
 #pragma unroll
@@ -185,7 +187,7 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
 #pragma unroll
             for (int i = 0; i < N; ++i) dot = fmaf(gM[i][j], B[i][j], dot);
 #pragma unroll
-            for (int i = 0; i < N; ++i) gM[i][j] = (gM[i][j] - dot) / cs[j];
+            for (int i = 0; i < N; ++i) gM[i][j] = (gM[i][j] - dot) * cs[j];
         }
     }
 #pragma unroll
@@ -216,7 +218,9 @@ bwd_dx_dphi_kernel(const T* __restrict__ X, const T* __restrict__ dY, const T* _
                    int tpg, T* __restrict__ dX, float* __restrict__ part) {
     constexpr int M = N * N + 2 * N;
     constexpr int CS = DX_THREADS / N >= 256 ? 256 : (DX_THREADS / N >= 128 ? 128 : 64);
-    __shared__ float sG[TB][M], sH[TB][M], sB[TB];
+    constexpr int MP = (M + 3) / 4 * 4;             // G rows padded for 16-byte reads
+    __shared__ __align__(16) float sG[TB][MP];
+    __shared__ float sH[TB][M], sB[TB];
     const int i = threadIdx.x / CS;
     const int c = blockIdx.x * CS + (threadIdx.x % CS);
     const bool active = i < N && c < d;
@@ -241,19 +245,41 @@ bwd_dx_dphi_kernel(const T* __restrict__ X, const T* __restrict__ dY, const T* _
         for (int u = threadIdx.x; u < nb; u += blockDim.x) sB[u] = beta[tb + u];
         __syncthreads();
         if (!active) continue;
-        for (int u = 0; u < nb; ++u) {
-            const int64_t t = tb + u;
-            const float v = to_f32(X[t * K + k]);
-            float pg = 0.f;
+        // UN tokens at a time: all their loads are issued before any of them is used
+        for (int u0 = 0; u0 < nb; u0 += UN) {
+            float v[UN], xi[UN], y[UN][N];
 #pragma unroll
-            for (int j = 0; j < M; ++j) {
-                acc[j] = fmaf(v, sG[u][j], acc[j]);
-                pg = fmaf(prow[j], sG[u][j], pg);
+            for (int q = 0; q < UN; ++q) {
+                const int64_t t = tb + (u0 + q < nb ? u0 + q : nb - 1);
+                v[q] = to_f32(X[t * K + k]);
+                xi[q] = to_f32(dx[t * d + c]);
+#pragma unroll
+                for (int p = 0; p < N; ++p) y[q][p] = to_f32(dY[t * K + (int64_t)p * d + c]);
             }
-            float g = sH[u][i] * to_f32(dx[t * d + c]) + pg - sB[u] * v;
 #pragma unroll
-            for (int q = 0; q < N; ++q) g = fmaf(sH[u][N + q * N + i], to_f32(dY[t * K + (int64_t)q * d + c]), g);
-            store_elem(&dX[t * K + k], g);
+            for (int q = 0; q < UN; ++q) {
+                const int u = u0 + q;
+                if (u < nb) {
+                    float pg = 0.f;
+#pragma unroll
+                    for (int j4 = 0; j4 < MP / 4; ++j4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(&sG[u][4 * j4]);
+                        const float ge[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 4 * j4 + e;
+                            if (j < M) {
+                                acc[j] = fmaf(v[q], ge[e], acc[j]);
+                                pg = fmaf(prow[j], ge[e], pg);
+                            }
+                        }
+                    }
+                    float g = sH[u][i] * xi[q] + pg - sB[u] * v[q];
+#pragma unroll
+                    for (int p = 0; p < N; ++p) g = fmaf(sH[u][N + p * N + i], y[q][p], g);
+                    store_elem(&dX[(tb + u) * K + k], g);
+                }
+            }
         }
     }
     if (active) {
