@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         s = lib.mhc_status_string(code)
         assert s and s.decode() != "unknown status"
     assert lib.mhc_status_string(99).decode() == "unknown status"
@@ -98,3 +98,39 @@ def test_binding_refuses_host_tensors():
 def test_path_query_on_cpu_host(lib):
     # With no usable GPU the query answers the generic path and launches nothing.
     assert lib.mhc_pre_path_for(16, 4, 64, 0) == mhc.PRE_GENERIC
+
+
+def _bwd(lib, X=A, F=A + 0x1000000, phi=A + 0x2000000, bp=A + 0x3000000, bq=A + 0x3000100,
+         br=A + 0x3000200, H=A + 0x4000000, h=A + 0x5000000, T=4, n=4, d=64, t_max=20, dt=1,
+         dY=A + 0x6000000, dx=A + 0x7000000, dX=A + 0x8000000, dF=A + 0x9000000,
+         dphi=A + 0xA000000, dbp=A + 0xB000000, dbq=A + 0xB000100, dbr=A + 0xB000200,
+         dal=A + 0xB000400, ws=A + 0xC000000, wsb=1 << 24):
+    return lib.mhc_backward(X, F, phi, bp, bq, br, 0.01, 0.01, 0.01, H, h, T, n, d, 1e-20, t_max,
+                            dt, dY, dx, dX, dF, dphi, dbp, dbq, dbr, dal, ws, wsb, None)
+
+
+def test_backward_validation(lib):
+    assert lib.mhc_backward_workspace_bytes(4, 4, 64) > 0
+    assert lib.mhc_backward_workspace_bytes(4, 5, 64) == 0          # n > 4: not supported
+    assert _bwd(lib, n=5) == 5 and _bwd(lib, n=0) == 2
+    assert _bwd(lib, t_max=-1) == 2 and _bwd(lib, dt=3) == 4
+    assert _bwd(lib, X=0) == 1 and _bwd(lib, ws=0) == 1 and _bwd(lib, phi=0) == 1
+    assert _bwd(lib, dal=0) == 1
+    assert _bwd(lib, X=A + 2) == 3                   # 16-byte alignment for the vector loads
+    assert _bwd(lib, d=60) == 3                      # 120-byte rows are not 16-byte multiples
+    assert _bwd(lib, ws=A + 0xC000010) == 3          # workspace: 256-byte alignment
+    need = lib.mhc_backward_workspace_bytes(4, 4, 64)
+    assert _bwd(lib, wsb=need - 1) == 8
+    assert _bwd(lib, dX=A + 64) == 7                 # dX overlaps X
+    assert _bwd(lib, dphi=A + 0xC000000) == 7        # dphi overlaps the workspace
+    assert _bwd(lib, dF=A + 0x6000000) == 7          # dF_out overlaps dX_out
+
+
+def test_pre_train_validation(lib):
+    def pre_train(h=A + 0x5000000, H=A + 0x4000000, T=4):
+        return lib.mhc_pre_train(A, A + 0x1000000, A + 0x2000000, A + 0x2000100, A + 0x2000200,
+                                 0.01, 0.01, 0.01, T, 4, 64, 1e-20, 20, 1, A + 0x3000000, H, h, None)
+    assert pre_train(T=0) == 0
+    assert pre_train(h=0) == 1
+    assert pre_train(h=A + 0x5000002) == 3
+    assert pre_train(h=A + 0x4000000) == 7           # h overlaps H
