@@ -180,6 +180,40 @@ mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, cons
                         float* db_res, float* dalpha, void* workspace, size_t workspace_bytes,
                         mhc_stream_t stream);
 
+/* Size of the fixed scratch array mhc_backward_noalloc works in: 32 MiB. */
+#define MHC_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * mhc_backward_noalloc -- mhc_backward without a caller-provided workspace, for callers
+ * that cannot allocate device memory: code that only receives device pointers from a host
+ * framework which owns every allocation through its own memory pool, or a call site where
+ * a cudaMalloc (which can synchronise the device) is not allowed.  The paper has no
+ * counterpart to this; it is a library convenience.
+ *
+ * Same arguments, results and errors as mhc_backward, minus the workspace pair.  The
+ * workspace is a fixed array of MHC_NOALLOC_SCRATCH_BYTES bytes inside the library's device
+ * image: every device on which the library's code is loaded holds it until the process
+ * exits, and the call itself allocates nothing (no cudaMalloc, no cudaFree).
+ *   - Sizes whose mhc_backward_workspace_bytes(T, n, d) exceeds MHC_NOALLOC_SCRATCH_BYTES
+ *     are rejected with MHC_ERR_WORKSPACE, launching nothing (T = 16384, n = 4, d = 4096
+ *     needs 30.0 MB and fits).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the one array, which keeps whatever the last call left
+ *     in it.  Nothing in it needs to start at zero (every kernel writes its part before
+ *     reading it), but calls that overlap on the GPU -- on different streams, or from
+ *     different host threads -- race on it: order them.
+ */
+mhc_status mhc_backward_noalloc(const void* X, const void* F_out, const float* phi,
+                                const float* b_pre, const float* b_post, const float* b_res,
+                                float alpha_pre, float alpha_post, float alpha_res,
+                                const float* H, const float* h, int64_t T, int n, int d,
+                                float eps, int t_max, mhc_dtype dt, const void* dX_out,
+                                const void* dx_in, void* dX, void* dF_out, float* dphi,
+                                float* db_pre, float* db_post, float* db_res, float* dalpha,
+                                mhc_stream_t stream);
+
 /*
  * mhc_device_status -- read and clear the device-side status word of the tensor-core
  * kernel.  Its waits between warps and between the CTAs of a cluster are bounded in

@@ -24,7 +24,8 @@ import os
 import threading
 
 __all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_post", "mhc_backward",
-           "mhc_backward_workspace_bytes", "mhc_pre_path_for", "mhc_device_status",
+           "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
+           "mhc_pre_path_for", "mhc_device_status",
            "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
@@ -33,6 +34,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmhc_b200.so")
 
 MHC_F32, MHC_BF16 = 0, 1
+NOALLOC_SCRATCH_BYTES = 32 << 20      # the fixed scratch array of mhc_backward_noalloc
 PRE_AUTO, PRE_GENERIC, PRE_CLUSTER_TC = 0, 1, 2
 _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN",
            4: "MHC_ERR_DTYPE", 5: "MHC_ERR_UNSUPPORTED", 6: "MHC_ERR_CUDA", 7: "MHC_ERR_ALIAS",
@@ -40,7 +42,8 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
 
 # Every function include/mhc.h declares.
 EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
-                    "mhc_backward_workspace_bytes", "mhc_backward", "mhc_status_string",
+                    "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
+                    "mhc_status_string",
                     "mhc_last_error", "mhc_device_status")
 
 _lock = threading.Lock()
@@ -82,6 +85,8 @@ def load_library():
         lib.mhc_backward.argtypes = ([vp, vp, fp, fp, fp, fp, cf, cf, cf, fp, fp, i64, ci, ci, cf, ci, ci,
                                       vp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ctypes.c_size_t, vp])
         lib.mhc_backward.restype = ci
+        lib.mhc_backward_noalloc.argtypes = lib.mhc_backward.argtypes[:-3] + [vp]
+        lib.mhc_backward_noalloc.restype = ci
         lib.mhc_pre_path_for.argtypes = [i64, ci, ci, ci]
         lib.mhc_pre_path_for.restype = ci
         lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
@@ -252,6 +257,35 @@ def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alp
                               p["dX"], p["dF_out"], q["dphi"], q["db_pre"], q["db_post"],
                               q["db_res"], q["dalpha"], ws, nbytes, _stream(stream, dev))
     _check(st, "mhc_backward")
+
+
+def mhc_backward_noalloc(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+                         eps, t_max, H, h, dX_out, dx_in, dX, dF_out, dphi, db_pre, db_post,
+                         db_res, dalpha, stream=None):
+    """mhc_backward for callers that cannot allocate device memory: the same gradients, with
+    the workspace in the library's fixed NOALLOC_SCRATCH_BYTES array instead of a caller
+    buffer.  Raises MhcError(MHC_ERR_WORKSPACE) for sizes that need more.  All calls on a
+    device share that array, so calls that overlap on the GPU must be ordered."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    f32 = torch.float32
+    dt = X.dtype
+    p = {k: _ptr(v, k, dt, dev) for k, v in dict(X=X, F_out=F_out, dX_out=dX_out, dx_in=dx_in,
+                                                  dX=dX, dF_out=dF_out).items()}
+    q = {k: _ptr(v, k, f32, dev) for k, v in dict(phi=phi, b_pre=b_pre, b_post=b_post, b_res=b_res,
+                                                   H=H, h=h, dphi=dphi, db_pre=db_pre,
+                                                   db_post=db_post, db_res=db_res,
+                                                   dalpha=dalpha).items()}
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_backward_noalloc(p["X"], p["F_out"], q["phi"], q["b_pre"], q["b_post"],
+                                      q["b_res"], float(alpha_pre), float(alpha_post),
+                                      float(alpha_res), q["H"], q["h"], T, n, d, float(eps),
+                                      int(t_max), _dt(X), p["dX_out"], p["dx_in"], p["dX"],
+                                      p["dF_out"], q["dphi"], q["db_pre"], q["db_post"],
+                                      q["db_res"], q["dalpha"], _stream(stream, dev))
+    _check(st, "mhc_backward_noalloc")
 
 
 def mhc_device_status() -> int:

@@ -20,6 +20,9 @@ static mhc_status cuda_fail(cudaError_t e, const char* where) {
     return MHC_ERR_CUDA;
 }
 
+// Records a CUDA error for mhc_last_error and returns MHC_ERR_CUDA (for other C-ABI files).
+mhc_status report_cuda_error(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+
 cudaError_t device_info(DeviceInfo* out) {
     constexpr int kMaxDev = 64;
     static DeviceInfo cache[kMaxDev];
