@@ -13,6 +13,8 @@ What each function follows (page title, section / equation):
                  page's HC update equation.
   * mhc_projection -- the normalised projection h of the same page's rmsnorm and
                  projection equations (what the training forward saves for the backward).
+  * amax_gain -- the Amax Gain Magnitude of composite residual maps ("DeepSeek-V4/mhc"
+                 page, stability paragraph; slavadubrov.com numpy demo).
   * mhc_backward -- reverse mode of pre + post (the chain rule through the steps above,
                  last step first; the Sinkhorn rounds recomputed from the logits).
 
@@ -72,6 +74,8 @@ def _load():
                                                  ctypes.c_double, ctypes.c_int] + [_dp] * 9 +
                                                 [ctypes.c_int])
             lib.oracle_mhc_backward.restype = None
+            lib.oracle_amax_gain.argtypes = [_dp, ctypes.c_int, ctypes.c_long, ctypes.c_int, _dp]
+            lib.oracle_amax_gain.restype = None
             lib.oracle_threads_used.argtypes = [ctypes.c_int]
             lib.oracle_threads_used.restype = ctypes.c_int
             _lib = lib
@@ -156,6 +160,18 @@ def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alp
                                 _p(out["dalpha"]), int(nthreads))
     out["db_res"] = out["db_res"].reshape(n, n)
     return out
+
+
+def amax_gain(Hs) -> np.ndarray:
+    """Hs [L, T, n*n+2n] (L layers' coefficient rows) -> gain [L, T, 2]: the largest absolute
+    row sum (forward) and column sum (backward) of C_l = H_res,l ... H_res,1, every l."""
+    Hs = _c(Hs)
+    L, T, m = Hs.shape
+    n = int(round((-2 + np.sqrt(4 + 4 * m)) / 2))
+    assert n * n + 2 * n == m and n <= 8, m
+    g = np.empty((L, T, 2), np.float64)
+    _load().oracle_amax_gain(_p(Hs), L, T, n, _p(g))
+    return g
 
 
 def threads_used(nthreads: int) -> int:

@@ -356,3 +356,38 @@ void oracle_mhc_backward(const double* X, const double* F_out, const double* phi
     }
     free(part);
 }
+
+/* Amax Gain Magnitude of the composite residual maps ("DeepSeek-V4/mhc" page, the
+ * stability paragraph: the largest absolute row sum -- forward -- and column sum --
+ * backward -- of prod_{i=1..l} H_res of layer l+1-i; the slavadubrov.com article's numpy
+ * demo forms the same product as C_l = H_res,l C_{l-1}).  Hs [L, T, m] holds each layer's
+ * coefficient rows as written by the pre stage (H_res at offset n); gain [L, T, 2]
+ * receives (forward, backward) of C_l for every prefix l = 1..L. */
+void oracle_amax_gain(const double* Hs, int L, long T, int n, double* gain)
+{
+    const int m = n * n + 2 * n;
+    double C[64], P[64];
+    for (long t = 0; t < T; ++t) {
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) C[i * n + j] = (i == j) ? 1.0 : 0.0;
+        for (int l = 0; l < L; ++l) {
+            const double* A = Hs + ((long)l * T + t) * m + n;
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j) {
+                    double s = 0.0;
+                    for (int q = 0; q < n; ++q) s += A[i * n + q] * C[q * n + j];
+                    P[i * n + j] = s;
+                }
+            memcpy(C, P, sizeof(double) * (size_t)(n * n));
+            double fwd = 0.0, bwd = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double r = 0.0, c = 0.0;
+                for (int j = 0; j < n; ++j) { r += fabs(C[i * n + j]); c += fabs(C[j * n + i]); }
+                if (r > fwd) fwd = r;
+                if (c > bwd) bwd = c;
+            }
+            gain[((long)l * T + t) * 2 + 0] = fwd;
+            gain[((long)l * T + t) * 2 + 1] = bwd;
+        }
+    }
+}

@@ -76,6 +76,11 @@ void oracle_mhc_backward(const double* X, const double* F_out, const double* phi
                          double* db_pre, double* db_post, double* db_res, double* dalpha,
                          int nthreads);
 
+/* Amax Gain Magnitude of the composite residual maps C_l = H_res,l ... H_res,1 for every
+ * prefix l of a stack of L layers: Hs [L, T, m] (each layer's coefficient rows), gain
+ * [L, T, 2] = (largest absolute row sum, largest absolute column sum) of C_l.  n <= 8. */
+void oracle_amax_gain(const double* Hs, int L, long T, int n, double* gain);
+
 /* Number of OpenMP threads a parallel region with the given request uses. */
 int oracle_threads_used(int nthreads);
 
