@@ -43,7 +43,7 @@ FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
 # measured on; reported as null once that source changes.
 NCU_TRAFFIC = {
     # measured at T=8192 (X = 256 MiB, twice the L2) and scaled x2 to T=16384
-    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.178304 + 50.199296) * 2e6), "66d4bb37f6ae0b95"),
+    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.162176 + 50.852096) * 2e6), "36fc8e56023222c5"),
     ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.358144 + 213.037056) * 2e6), "96dbcd70460419e6"),
 }
 
@@ -524,6 +524,53 @@ def run_backward(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+def run_amax(args, rank, world, local_rank):
+    """The depth-stability diagnostic: mhc_amax_gain over the coefficient rows of L = 60
+    layers (the 27B model's depth) for T tokens at n = 4.  Prints one JSON line."""
+    import torch
+
+    import mhc_hyper_connections_b200 as mhc
+    from mhc_hyper_connections_b200 import dist as mdist
+    from mhc_hyper_connections_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.make_config(args.config)
+    T = args.tokens or w.T
+    n, L = w.n, 60
+    m = n * n + 2 * n
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + rank)
+    Hs = torch.rand(L, T, m, device=dev, generator=g)          # stand-in maps, fp32
+    gain = torch.empty(L, T, 2, device=dev)
+    for _ in range(args.warmup):
+        mhc.mhc_amax_gain(Hs, gain)
+    torch.cuda.synchronize()
+    K = args.steps
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        mhc.mhc_amax_gain(Hs, gain)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    ms = mdist.max_over_ranks(ms, device=dev)
+    by = L * T * (m * 4 + 8)
+    peak, peak_src = _hbm_peak()
+    gbs = by / (ms / 1e3 / K) / 1e9
+    line = {"metric": "mHC composite Amax gain (diagnostic): layer-tokens/s, L=60 n=4",
+            "value": L * T * K * world / (ms / 1e3), "unit": "layer-tokens/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"amax_L{L}_T{T}_n{n}", "L": L, "T": T, "n": n},
+            "roofline": {"kernel": "amax_gain_kernel", "bound": "hbm", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak, "traffic": None, "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": by},
+            "gpu_launches": K}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     from mhc_hyper_connections_b200 import workloads as wl
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
@@ -541,6 +588,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--amax", action="store_true",
+                    help="time the composite Amax gain diagnostic (mhc_amax_gain, 60 layers)")
     ap.add_argument("--backward", action="store_true",
                     help="time forward + backward steps (mhc_pre_train, mhc_post, mhc_backward)")
     args = ap.parse_args()
@@ -556,6 +605,8 @@ def main():
         return run_reference(args, rank, world)
     if args.backward:
         return run_backward(args, rank, world, local_rank)
+    if args.amax:
+        return run_amax(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 

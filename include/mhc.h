@@ -215,6 +215,22 @@ mhc_status mhc_backward_noalloc(const void* X, const void* F_out, const float* p
                                 mhc_stream_t stream);
 
 /*
+ * mhc_amax_gain -- the Amax Gain Magnitude of the composite residual maps of L consecutive
+ * layers ("DeepSeek-V4/mhc" page, stability paragraph; the slavadubrov.com article's numpy
+ * demo): for every token and every prefix l = 1..L of the stack,
+ *   C_l = H_res(layer l) . H_res(layer l-1) ... H_res(layer 1)
+ *   gain[l-1, t, 0] = max_i sum_j |C_l[i][j]|   (forward: largest absolute row sum)
+ *   gain[l-1, t, 1] = max_j sum_i |C_l[i][j]|   (backward: largest absolute column sum)
+ * A diagnostic of depth-wise stability, not part of the layer's hot path.
+ * Inputs : H_layers [L, T, m] fp32, the coefficient rows mhc_pre wrote for each layer,
+ *          stacked (layer l at H_layers + l*T*m); 1 <= n <= 8, L >= 0, T >= 0.
+ * Output : gain [L, T, 2] fp32, written in place; may not overlap H_layers.
+ * L == 0 or T == 0 returns MHC_OK and launches nothing.
+ */
+mhc_status mhc_amax_gain(const float* H_layers, int L, int64_t T, int n, float* gain,
+                         mhc_stream_t stream);
+
+/*
  * mhc_device_status -- read and clear the device-side status word of the tensor-core
  * kernel.  Its waits between warps and between the CTAs of a cluster are bounded in
  * time (1 s each); a wait that expires makes the kernel stop early, leaving its outputs

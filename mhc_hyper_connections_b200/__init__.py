@@ -25,7 +25,7 @@ import threading
 
 __all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_post", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
-           "mhc_pre_path_for", "mhc_device_status",
+           "mhc_amax_gain", "mhc_pre_path_for", "mhc_device_status",
            "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
@@ -43,7 +43,7 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
 # Every function include/mhc.h declares.
 EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
-                    "mhc_status_string",
+                    "mhc_amax_gain", "mhc_status_string",
                     "mhc_last_error", "mhc_device_status")
 
 _lock = threading.Lock()
@@ -87,6 +87,8 @@ def load_library():
         lib.mhc_backward.restype = ci
         lib.mhc_backward_noalloc.argtypes = lib.mhc_backward.argtypes[:-3] + [vp]
         lib.mhc_backward_noalloc.restype = ci
+        lib.mhc_amax_gain.argtypes = [fp, ci, i64, ci, fp, vp]
+        lib.mhc_amax_gain.restype = ci
         lib.mhc_pre_path_for.argtypes = [i64, ci, ci, ci]
         lib.mhc_pre_path_for.restype = ci
         lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
@@ -286,6 +288,24 @@ def mhc_backward_noalloc(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_p
                                       p["dF_out"], q["dphi"], q["db_pre"], q["db_post"],
                                       q["db_res"], q["dalpha"], _stream(stream, dev))
     _check(st, "mhc_backward_noalloc")
+
+
+def mhc_amax_gain(H_layers, gain, stream=None):
+    """Amax Gain Magnitude of composite residual maps: H_layers [L, T, n*n+2n] fp32 (each
+    layer's H from mhc_pre, stacked) -> gain [L, T, 2] fp32 = (largest absolute row sum,
+    largest absolute column sum) of H_res(l) ... H_res(1) for every prefix l."""
+    import torch
+    L, T, m = H_layers.shape
+    n = int(round(((4 + 4 * m) ** 0.5 - 2) / 2))
+    if n * n + 2 * n != m or tuple(gain.shape) != (L, T, 2):
+        raise ValueError("mhc_amax_gain: H_layers [L, T, n*n+2n] and gain [L, T, 2]")
+    dev = H_layers.device
+    hp = _ptr(H_layers, "H_layers", torch.float32, dev)
+    gp = _ptr(gain, "gain", torch.float32, dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_amax_gain(hp, L, T, n, gp, _stream(stream, dev))
+    _check(st, "mhc_amax_gain")
 
 
 def mhc_device_status() -> int:

@@ -92,6 +92,9 @@ struct BwdLayout {
     int64_t tokens_per_group;
 };
 BwdLayout backward_layout(int64_t T, int n, int d);
+
+// Amax Gain Magnitude of composite residual maps (diagnostics.cu).
+cudaError_t launch_amax_gain(const float* Hs, int L, int64_t T, int n, float* gain, cudaStream_t s);
 cudaError_t launch_backward(const BwdArgs& a);
 
 }  // namespace mhc

@@ -277,6 +277,20 @@ mhc_status mhc_post(const void* X, const void* F_out, const float* H, int64_t T,
     return MHC_OK;
 }
 
+mhc_status mhc_amax_gain(const float* H_layers, int L, int64_t T, int n, float* gain,
+                         mhc_stream_t stream) {
+    if (n < 1 || n > 8 || L < 0 || T < 0) return MHC_ERR_SHAPE;
+    const int m = n * n + 2 * n;
+    if (L > 0 && T > (((int64_t)1 << 58) / ((int64_t)L * m))) return MHC_ERR_SHAPE;
+    if (L == 0 || T == 0) return MHC_OK;
+    if (!H_layers || !gain) return MHC_ERR_NULL;
+    if (!aligned(H_layers, 4) || !aligned(gain, 4)) return MHC_ERR_ALIGN;
+    if (overlaps(gain, (size_t)L * T * 8, H_layers, (size_t)L * T * m * 4)) return MHC_ERR_ALIAS;
+    cudaError_t e = launch_amax_gain(H_layers, L, T, n, gain, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "mhc_amax_gain");
+    return MHC_OK;
+}
+
 const char* mhc_status_string(mhc_status s) {
     switch (s) {
         case MHC_OK: return "ok";

@@ -134,3 +134,13 @@ def test_pre_train_validation(lib):
     assert pre_train(h=0) == 1
     assert pre_train(h=A + 0x5000002) == 3
     assert pre_train(h=A + 0x4000000) == 7           # h overlaps H
+
+
+def test_amax_gain_validation(lib):
+    assert lib.mhc_amax_gain(A, 0, 5, 4, A + 0x1000000, None) == 0      # L = 0: nothing to do
+    assert lib.mhc_amax_gain(A, 3, 0, 4, A + 0x1000000, None) == 0      # T = 0
+    assert lib.mhc_amax_gain(A, 3, 5, 9, A + 0x1000000, None) == 2
+    assert lib.mhc_amax_gain(A, -1, 5, 4, A + 0x1000000, None) == 2
+    assert lib.mhc_amax_gain(0, 3, 5, 4, A + 0x1000000, None) == 1
+    assert lib.mhc_amax_gain(A, 3, 5, 4, A + 2, None) == 3
+    assert lib.mhc_amax_gain(A, 3, 5, 4, A + 64, None) == 7             # gain overlaps H_layers
