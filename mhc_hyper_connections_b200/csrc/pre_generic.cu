@@ -2,7 +2,8 @@
 //
 // Per CTA a tile of TT tokens:
 //   1. K loop (K = n*d): stage X[tile, k0:k0+KC] (as fp32) and phi[k0:k0+KC, :] in shared
-//      memory; accumulate the projection h = v . phi (fp32) and the sum of squares of v.
+//      memory; accumulate the projection h = v . phi (fp32; each thread a TM-token by
+//      ceil(m/32)-column register tile) and the sum of squares of v.
 //   2. One thread per token turns h into [H_pre | H_res | H_post] ("DeepSeek-V4/mhc",
 //      equations rmsnorm, a/b/c-tilde, gate, sinkhorn) and writes H.
 //   3. x_in = sum_i H_pre[i] X[t, i, :] (slavadubrov.com Eq. 3, read map on raw X).
@@ -14,9 +15,11 @@
 namespace mhc {
 namespace {
 
-constexpr int TT = 16;        // tokens per CTA
-constexpr int KC = 64;        // K chunk staged per step
+constexpr int TT = 32;        // tokens per CTA
+constexpr int KC = 32;        // K chunk staged per step
 constexpr int THREADS = 256;
+constexpr int TM = 4;         // tokens of a thread's projection micro-tile
+constexpr int JS = THREADS / (TT / TM);     // column groups: thread columns j = jg + JS * q
 
 template <int N, typename T>
 __global__ void __launch_bounds__(THREADS)
@@ -27,9 +30,10 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
                    float* __restrict__ H, float* __restrict__ h_out)
 {
     constexpr int M = N * N + 2 * N;
-    constexpr int NO = (TT * M + THREADS - 1) / THREADS;   // projection outputs per thread
+    constexpr int TJ = (M + JS - 1) / JS;              // columns per thread
+    constexpr int SPT = KC * TT / THREADS;             // X elements staged per thread
     __shared__ float xs[TT][KC + 1];
-    __shared__ float ps[KC][M];
+    __shared__ float ps[KC][JS * TJ];                  // columns past M hold zeros
     __shared__ float hs[TT][M];
     __shared__ float ss_s[TT];
     __shared__ float hpre_s[TT][N];
@@ -37,18 +41,21 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
     const int K = N * d;
     const int64_t t0 = (int64_t)blockIdx.x * TT;
     const int tid = threadIdx.x;
+    const int tg = tid / JS, jg = tid % JS;             // micro-tile: tokens tg*TM.., columns jg + JS*q
 
-    float acc[NO];
+    float acc[TM][TJ];
 #pragma unroll
-    for (int r = 0; r < NO; ++r) acc[r] = 0.f;
-    float ssq = 0.f;                                  // partial sum of squares, token tid/16
-    const int my_t = tid / (THREADS / TT);            // 16 threads per token when staging
-    const int my_k0 = (tid % (THREADS / TT)) * (KC * TT / THREADS);
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int q = 0; q < TJ; ++q) acc[a][q] = 0.f;
+    float ssq = 0.f;                                  // partial sum of squares of token my_t
+    const int my_t = tid / (THREADS / TT);            // THREADS / TT threads per token when staging
+    const int my_k0 = (tid % (THREADS / TT)) * SPT;
     const int64_t my_tok = t0 + my_t;
 
     for (int k0 = 0; k0 < K; k0 += KC) {
 #pragma unroll
-        for (int u = 0; u < KC * TT / THREADS; ++u) {
+        for (int u = 0; u < SPT; ++u) {
             const int kk = my_k0 + u;
             const int k = k0 + kk;
             float v = 0.f;
@@ -56,34 +63,37 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
             xs[my_t][kk] = v;
             ssq = fmaf(v, v, ssq);
         }
-        for (int e = tid; e < KC * M; e += THREADS) {
-            const int kk = e / M, j = e - kk * M;
+        for (int e = tid; e < KC * JS * TJ; e += THREADS) {
+            const int kk = e / (JS * TJ), j = e - kk * (JS * TJ);
             const int k = k0 + kk;
-            ps[kk][j] = (k < K) ? phi[(int64_t)k * M + j] : 0.f;
+            ps[kk][j] = (k < K && j < M) ? phi[(int64_t)k * M + j] : 0.f;
         }
         __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < KC; ++kk) {
+            float xv[TM], pv[TJ];
 #pragma unroll
-        for (int r = 0; r < NO; ++r) {
-            const int o = tid + THREADS * r;
-            if (o < TT * M) {
-                const int t = o / M, j = o - t * M;
-                float a = acc[r];
-#pragma unroll 8
-                for (int kk = 0; kk < KC; ++kk) a = fmaf(xs[t][kk], ps[kk][j], a);
-                acc[r] = a;
-            }
+            for (int a = 0; a < TM; ++a) xv[a] = xs[tg * TM + a][kk];
+#pragma unroll
+            for (int q = 0; q < TJ; ++q) pv[q] = ps[kk][jg + JS * q];
+#pragma unroll
+            for (int a = 0; a < TM; ++a)
+#pragma unroll
+                for (int q = 0; q < TJ; ++q) acc[a][q] = fmaf(xv[a], pv[q], acc[a][q]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int r = 0; r < NO; ++r) {
-        const int o = tid + THREADS * r;
-        if (o < TT * M) hs[o / M][o % M] = acc[r];
-    }
-    // sum of squares: the 16 threads of a token are one half-warp
+    for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
-    if ((tid & 15) == 0) ss_s[my_t] = ssq;
+        for (int q = 0; q < TJ; ++q) {
+            const int j = jg + JS * q;
+            if (j < M) hs[tg * TM + a][j] = acc[a][q];
+        }
+    // sum of squares: the THREADS / TT threads of a token are consecutive lanes
+#pragma unroll
+    for (int off = THREADS / TT / 2; off > 0; off >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+    if ((tid % (THREADS / TT)) == 0) ss_s[my_t] = ssq;
     __syncthreads();
 
     if (tid < TT && t0 + tid < Tn) {
