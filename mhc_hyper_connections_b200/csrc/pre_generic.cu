@@ -53,22 +53,38 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
     const int my_k0 = (tid % (THREADS / TT)) * SPT;
     const int64_t my_tok = t0 + my_t;
 
+    // chunk k0's X and phi values travel through registers: the next chunk's loads are in
+    // flight while this chunk is multiplied
+    constexpr int PPT = (KC * JS * TJ + THREADS - 1) / THREADS;   // phi values staged per thread
+    float xr[SPT], pr[PPT];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int u = 0; u < SPT; ++u) {
+            const int k = k0 + my_k0 + u;
+            xr[u] = (my_tok < Tn && k < K) ? to_f32(X[my_tok * K + k]) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < PPT; ++r) {
+            const int e = tid + THREADS * r;
+            const int kk = e / (JS * TJ), j = e - kk * (JS * TJ);
+            const int k = k0 + kk;
+            pr[r] = (e < KC * JS * TJ && k < K && j < M) ? phi[(int64_t)k * M + j] : 0.f;
+        }
+    };
+    fetch(0);
     for (int k0 = 0; k0 < K; k0 += KC) {
 #pragma unroll
         for (int u = 0; u < SPT; ++u) {
-            const int kk = my_k0 + u;
-            const int k = k0 + kk;
-            float v = 0.f;
-            if (my_tok < Tn && k < K) v = to_f32(X[my_tok * K + k]);
-            xs[my_t][kk] = v;
-            ssq = fmaf(v, v, ssq);
+            xs[my_t][my_k0 + u] = xr[u];
+            ssq = fmaf(xr[u], xr[u], ssq);
         }
-        for (int e = tid; e < KC * JS * TJ; e += THREADS) {
-            const int kk = e / (JS * TJ), j = e - kk * (JS * TJ);
-            const int k = k0 + kk;
-            ps[kk][j] = (k < K && j < M) ? phi[(int64_t)k * M + j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < PPT; ++r) {
+            const int e = tid + THREADS * r;
+            if (e < KC * JS * TJ) ps[e / (JS * TJ)][e % (JS * TJ)] = pr[r];
         }
         __syncthreads();
+        if (k0 + KC < K) fetch(k0 + KC);
 #pragma unroll 4
         for (int kk = 0; kk < KC; ++kk) {
             float xv[TM], pv[TJ];
