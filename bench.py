@@ -403,7 +403,9 @@ def run_ours(args, rank, world, local_rank):
 def run_backward(args, rank, world, local_rank):
     """Forward + backward steps (mhc_pre_train, mhc_post, mhc_backward) on one batch: the
     backward workload (T=16384, n=4, d=4096, bf16 with outlier channels, upstream gradients
-    dX_out and dx_in ~ N(0,1) in bf16).  Prints one JSON line."""
+    dX_out and dx_in ~ N(0,1) in bf16).  Under torchrun every rank runs its own batch and
+    the parameter gradients are all-reduced each step (data parallel).  Prints one JSON
+    line."""
     import numpy as np
     import torch
 
@@ -455,9 +457,14 @@ def run_backward(args, rank, world, local_rank):
     def post():
         mhc.mhc_post(X, F, H, Y)
 
+    pgrads = dict(dphi=dphi, db_pre=db_pre, db_post=db_post, db_res=db_res, dalpha=dalpha)
+
     def bwd():
         mhc.mhc_backward(X, F, phi, b_pre, b_post, b_res, *sa, H, h, dY, dxi, dX, dF, dphi,
                          db_pre, db_post, db_res, dalpha, ws)
+        # data-parallel step: the parameter gradients are summed over the ranks (NCCL); a
+        # no-op on one GPU
+        mdist.allreduce_param_grads(pgrads)
 
     for _ in range(args.warmup):
         fwd(); post(); bwd()
@@ -500,6 +507,7 @@ def run_backward(args, rank, world, local_rank):
         "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": args.config + "+backward", "T": T, "n": n, "d": d,
+                   "parallelism": f"dp{world} (token batches per rank, parameter-gradient all-reduce)",
                    "upstream": "dX_out, dx_in ~ N(0,1), stored like X",
                    "l2": "inputs larger than L2, no flush"},
         "kernels": {"pre_train": {"ms": st[0], "bytes_per_launch": by_pre * T,

@@ -1,6 +1,8 @@
 """The multi-rank path on CPU: world size 2 over gloo (127.0.0.1).  Each rank runs the fp64
 oracle on its token shard; the shards reassemble to the single-process result (tokens are
-independent), and the timing reduction takes the max over ranks."""
+independent), and the timing reduction takes the max over ranks.  For the backward, each
+rank's parameter gradients over its shard, summed across ranks by allreduce_param_grads,
+equal the gradients over all tokens."""
 import os
 import socket
 
@@ -77,3 +79,56 @@ def test_two_gloo_ranks_reassemble_and_reduce(tmp_path):
     np.testing.assert_array_equal(np.concatenate([p["y"] for p in parts]), y)
     for r in range(world):
         assert float(np.load(tmp_path / f"m{r}.npy")[0]) == 15.0
+
+
+def _bwd_worker(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from mhc_hyper_connections_b200 import workloads as wl
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w, dY, dx = _bwd_problem()
+        a, b = mdist.token_shard(w.T, rank, world)
+        sub = w.tokens(np.arange(a, b))
+        s = w.scalars()
+        g = oracle.mhc_backward(sub.values(sub.X), sub.values(sub.F_out), sub.phi, sub.b_pre,
+                                sub.b_post, sub.b_res, s["alpha_pre"], s["alpha_post"],
+                                s["alpha_res"], dY[a:b], dx[a:b], eps=s["eps"], t_max=s["t_max"])
+        tg = {k: torch.from_numpy(g[k]) for k in mdist.PARAM_GRADS}
+        mdist.allreduce_param_grads(tg)
+        np.savez(os.path.join(out_dir, f"g{rank}.npz"), dX=g["dX"], dF_out=g["dF_out"],
+                 **{k: v.numpy() for k, v in tg.items()})
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _bwd_problem():
+    from mhc_hyper_connections_b200 import workloads as wl
+    w = wl.make_inputs(T=37, n=3, d=16, dtype="bf16", seed=8, alpha=0.4)
+    rng = np.random.default_rng(9)
+    return w, rng.normal(size=(w.T, w.n, w.d)), rng.normal(size=(w.T, w.d))
+
+
+def test_two_gloo_ranks_sum_the_parameter_gradients(tmp_path):
+    import oracle
+    oracle.build()
+    world, port = 2, _free_port()
+    mp.start_processes(_bwd_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    parts = [np.load(tmp_path / f"g{r}.npz") for r in range(world)]
+    w, dY, dx = _bwd_problem()
+    s = w.scalars()
+    ref = oracle.mhc_backward(w.values(w.X), w.values(w.F_out), w.phi, w.b_pre, w.b_post, w.b_res,
+                              s["alpha_pre"], s["alpha_post"], s["alpha_res"], dY, dx,
+                              eps=s["eps"], t_max=s["t_max"])
+    np.testing.assert_array_equal(np.concatenate([p["dX"] for p in parts]), ref["dX"])
+    np.testing.assert_array_equal(np.concatenate([p["dF_out"] for p in parts]), ref["dF_out"])
+    for k in mdist.PARAM_GRADS:
+        for p in parts:                     # every rank holds the whole job's gradient
+            np.testing.assert_allclose(p[k].reshape(ref[k].shape), ref[k], rtol=1e-12, atol=1e-14)
+    assert mdist.allreduce_param_grads({}) is None    # no process group here: a no-op
