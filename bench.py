@@ -45,6 +45,8 @@ NCU_TRAFFIC = {
     # measured at T=8192 (X = 256 MiB, twice the L2) and scaled x2 to T=16384
     ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.162176 + 50.852096) * 2e6), "36fc8e56023222c5"),
     ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.358144 + 213.037056) * 2e6), "96dbcd70460419e6"),
+    # the six launches of one mhc_backward call, captured at T=16384 itself
+    ("backward", "bf16_T16384_n4_d4096_outliers"): (2595292928 + 615071232, "168cedaecef3c0ce"),
 }
 
 
@@ -326,8 +328,8 @@ def run_ours(args, rank, world, local_rank):
     dom = max(kern, key=lambda k: kern[k]["ms"])
     traffic = None
     rec = NCU_TRAFFIC.get((dom, args.config))
-    if rec and rec[1] == _src_sha(kern[dom]["source"]):
-        traffic = rec[0]
+    if rec and not args.tokens and rec[1] == _src_sha(kern[dom]["source"]):
+        traffic = rec[0]                       # the capture is of the full token count
     achieved = kern[dom]["gbs"]
     roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
@@ -501,6 +503,9 @@ def run_backward(args, rank, world, local_rank):
     bw_gbs = by_bwd * T / (st[2] / 1e3) / 1e9
     step_bytes = (by_pre + by_post + by_bwd) * T
     step_gbs = step_bytes / (ms_total / 1e3 / K) / 1e9       # per GPU: each processes T tokens
+    bwd_src = "mhc_hyper_connections_b200/csrc/backward.cu"
+    rec = NCU_TRAFFIC.get(("backward", args.config))
+    traffic = rec[0] if (rec and not args.tokens and rec[1] == _src_sha(bwd_src)) else None
     line = {
         "metric": "mHC forward+backward tokens/s (pre_train + post + backward), n=4 d=4096 bf16",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -516,9 +521,9 @@ def run_backward(args, rank, world, local_rank):
                              "gbs": by_post * T / (st[1] / 1e3) / 1e9},
                     "backward": {"ms": st[2], "bytes_per_launch": by_bwd * T, "gbs": bw_gbs,
                                  "launches": 6,
-                                 "source": "mhc_hyper_connections_b200/csrc/backward.cu"}},
+                                 "source": bwd_src}},
         "roofline": {"kernel": "backward (6 launches)", "bound": "hbm", "achieved": bw_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": bw_gbs / peak, "traffic": None,
+                     "peak": peak, "unit": "GB/s", "frac": bw_gbs / peak, "traffic": traffic,
                      "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": by_bwd * T},
         "hbm": {"step_bytes_per_token": by_pre + by_post + by_bwd, "gbs_per_gpu": step_gbs,
