@@ -45,8 +45,9 @@ NCU_TRAFFIC = {
     # measured at T=8192 (X = 256 MiB, twice the L2) and scaled x2 to T=16384
     ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.162176 + 50.852096) * 2e6), "36fc8e56023222c5"),
     ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.358144 + 213.037056) * 2e6), "96dbcd70460419e6"),
-    # the six launches of one mhc_backward call, captured at T=16384 itself
-    ("backward", "bf16_T16384_n4_d4096_outliers"): (2595292928 + 615071232, "168cedaecef3c0ce"),
+    # the six launches of one mhc_backward call, captured at T=16384 itself (on the file's
+    # previous hash 8883e6aea5058f0e: since then only its header comment changed)
+    ("backward", "bf16_T16384_n4_d4096_outliers"): (2595701760 + 615055104, "2fad304296d6ff37"),
 }
 
 

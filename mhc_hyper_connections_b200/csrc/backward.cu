@@ -19,8 +19,9 @@
 // Kernels, in launch order:
 //   K1 bwd_reduce   warp per token: the sums over channels (sum X^2, dH_pre, dH_res,
 //                   dH_post) into a workspace row, and dF_out
-//   K2 bwd_token    thread per token: gates, Sinkhorn backward (O(t_max^2) recomputed
-//                   half-steps, nothing stored), G = g / r and beta = (g . h) / (K r^2)
+//   K2 bwd_token    thread per token: gates, Sinkhorn backward (each round's input is
+//                   kept in shared memory, then the rounds run in reverse), G = g / r and
+//                   beta = (g . h) / (K r^2)
 //   K3 bwd_dx_dphi  CTA per (channel slice, token group): dX, and the group's partial dphi
 //                   (each thread keeps one phi row and one dphi row in registers)
 //   K4 reductions   dphi over the groups, db and dalpha over the tokens, all in a fixed
@@ -32,7 +33,8 @@ namespace mhc {
 namespace {
 
 constexpr int RED_THREADS = 256;
-constexpr int TOK_THREADS = 128;
+constexpr int TOK_THREADS = 32;     // K2: one warp per block spreads 16 K tokens over every SM
+constexpr int SK_SLOTS = 20;        // K2: Sinkhorn round inputs kept per token
 constexpr int DX_THREADS = 256;
 constexpr int TB = 32;               // tokens staged per batch in K3
 constexpr int UN = 8;                // tokens whose loads K3 has in flight at once
@@ -148,7 +150,13 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         const float s = 0.5f * H[t * M + N + N * N + i];
         out[N + N * N + i] = Rt[1 + N + N * N + i] * 2.f * s * (1.f - s);
     }
-    // Sinkhorn: M0 = exp(l_res); the backward of round s needs its input A, recomputed
+    // Sinkhorn: M0 = exp(l_res); the backward of round s needs that round's input A_s.
+    // The inputs of rounds 0, S, 2S, ... are kept in shared memory (this thread's column of
+    // ck), S = 1 while t_max <= SK_SLOTS; A_s is rebuilt by replaying rounds from the kept
+    // input at or below s.  That is t_max - 1 + t_max rounds for t_max <= SK_SLOTS instead of
+    // the t_max (t_max + 1) / 2 of replaying every A_s from M0.
+    __shared__ float ck[SK_SLOTS][N * N][TOK_THREADS];
+    const int lane = threadIdx.x;
     float M0[N][N], gM[N][N];
 #pragma unroll
     for (int i = 0; i < N; ++i)
@@ -157,13 +165,37 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
             M0[i][j] = expf(a_res * hh[N + i * N + j] + b_res[i * N + j]);
             gM[i][j] = Rt[1 + N + i * N + j];
         }
-    for (int s = t_max - 1; s >= 0; --s) {
+    // S >= t_max / SK_SLOTS, so every kept index k (k S < t_max) is below SK_SLOTS
+    const int S = t_max <= SK_SLOTS ? 1 : (t_max + SK_SLOTS - 1) / SK_SLOTS;
+    {
         float A[N][N], B[N][N], C[N][N], cs[N], rs[N];
 #pragma unroll
         for (int i = 0; i < N; ++i)
 #pragma unroll
             for (int j = 0; j < N; ++j) A[i][j] = M0[i][j];
-        for (int u = 0; u < s; ++u) {
+        for (int k = 0; k * S < t_max; ++k) {
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+#pragma unroll
+                for (int j = 0; j < N; ++j) ck[k][i * N + j][lane] = A[i][j];
+            if ((k + 1) * S >= t_max) break;
+            for (int v = 0; v < S; ++v) {
+                sk_round<N>(A, B, C, cs, rs);
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int j = 0; j < N; ++j) A[i][j] = C[i][j];
+            }
+        }
+    }
+    for (int s = t_max - 1; s >= 0; --s) {
+        float A[N][N], B[N][N], C[N][N], cs[N], rs[N];
+        const int k = s / S;
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+#pragma unroll
+            for (int j = 0; j < N; ++j) A[i][j] = ck[k][i * N + j][lane];
+        for (int u = k * S; u < s; ++u) {
             sk_round<N>(A, B, C, cs, rs);
 #pragma unroll
             for (int i = 0; i < N; ++i)

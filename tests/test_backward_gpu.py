@@ -9,6 +9,8 @@ checked entry by entry as |gpu - ref| <= rtol |ref| + atol * max|ref|:
   fp32 I/O     rtol 1e-4,            atol 1e-5
   bf16 I/O     dX, dF_out: rtol 2^-8 * 1.01, atol 2e-3; parameter gradients (fp32 sums over
                tokens of bf16-exact inputs): rtol 1e-3, atol 1e-4."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -121,6 +123,17 @@ def test_shapes(T, n, d, dt):
     w = wl.make_inputs(T=T, n=n, d=d, dtype=dt, seed=T * 7 + n * 3 + d, alpha=0.3)
     dY, dx = _upstream(w, T + d)
     check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"T{T} n{n} d{d} {dt}")
+
+
+@pytest.mark.parametrize("t_max,n", [(0, 4), (1, 4), (3, 3), (21, 4), (41, 2), (64, 4)])
+def test_sinkhorn_depths(t_max, n):
+    """Sinkhorn depths other than 20: none (H_res = exp of the logits), one round, and depths
+    past the 20 round inputs the backward keeps per token, where it keeps every 2nd, 3rd or
+    4th and replays the rounds in between."""
+    w = wl.make_inputs(T=70, n=n, d=40, dtype="bf16", seed=500 + t_max, alpha=0.3)
+    w = dataclasses.replace(w, t_max=t_max)
+    dY, dx = _upstream(w, 600 + t_max)
+    check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"t_max {t_max} n {n}")
 
 
 def test_headline_size_sampled_and_additive():
