@@ -13,8 +13,8 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    # A GPU test never silently passes on a box without a GPU: it is skipped with a reason
-    # here, and on a GPU machine the CUDA library must load or the test fails.
+    # A GPU test never silently passes on a machine without a GPU: it is skipped with a
+    # reason there, and on a machine with one the CUDA library must load or the test fails.
     try:
         import torch
         has_gpu = torch.cuda.is_available()
