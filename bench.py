@@ -193,36 +193,46 @@ def run_reference(args, rank, world):
     return 0
 
 
-def cpu_baseline(w, seconds=10.0, chunk=1024, max_passes=64):
+def cpu_baseline(w, seconds=10.0, chunk=1024, max_passes=64, single_seconds=3.0):
     """The oracle as it stands, on the host cores, over a bounded token sample: passes over
     the batch in chunks of `chunk` tokens (fp64 conversion outside the timed calls) until
-    about `seconds` of timed oracle work has accumulated."""
+    about `seconds` of timed oracle work has accumulated on all cores, then about
+    `single_seconds` more on one thread."""
     import numpy as np
 
     import oracle
     cores = os.cpu_count() or 1
     used = oracle.threads_used(cores)
     s = w.scalars()
-    done, t_sum, passes = 0, 0.0, 0
-    while t_sum < seconds and passes < max_passes:
-        for c0 in range(0, w.T, chunk):
-            sub = w.tokens(np.arange(c0, min(w.T, c0 + chunk)))
-            X = sub.values(sub.X)
-            F = sub.values(sub.F_out)
-            t0 = time.perf_counter()
-            _, H = oracle.mhc_pre(X, sub.phi, sub.b_pre, sub.b_post, sub.b_res, s["alpha_pre"],
-                                  s["alpha_post"], s["alpha_res"], eps=s["eps"], t_max=s["t_max"],
-                                  nthreads=cores)
-            oracle.mhc_post(X, F, H, nthreads=cores)
-            t_sum += time.perf_counter() - t0
-            done += sub.T
-            if t_sum >= seconds:
-                break
-        passes += 1
+
+    def timed(nthreads, budget):
+        done, t_sum, passes = 0, 0.0, 0
+        while t_sum < budget and passes < max_passes:
+            for c0 in range(0, w.T, chunk):
+                sub = w.tokens(np.arange(c0, min(w.T, c0 + chunk)))
+                X = sub.values(sub.X)
+                F = sub.values(sub.F_out)
+                t0 = time.perf_counter()
+                _, H = oracle.mhc_pre(X, sub.phi, sub.b_pre, sub.b_post, sub.b_res, s["alpha_pre"],
+                                      s["alpha_post"], s["alpha_res"], eps=s["eps"], t_max=s["t_max"],
+                                      nthreads=nthreads)
+                oracle.mhc_post(X, F, H, nthreads=nthreads)
+                t_sum += time.perf_counter() - t0
+                done += sub.T
+                if t_sum >= budget:
+                    break
+            passes += 1
+        return done, t_sum, passes
+
+    done, t_sum, passes = timed(cores, seconds)
+    one_done, one_t, _ = timed(1, single_seconds)
     return {"value": done / t_sum, "unit": "tokens/s", "cores": used, "kind": "oracle",
             "sample": f"{done} tokens ({passes} pass(es) over the {w.T}-token batch in "
                       f"{chunk}-token chunks), {t_sum:.1f} s of fp64 oracle time on {used} "
-                      f"OpenMP threads"}
+                      f"OpenMP threads",
+            "single_thread": {"value": one_done / one_t, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{one_done} tokens in {chunk}-token chunks from the "
+                                        f"start of the batch, {one_t:.1f} s on one thread"}}
 
 
 # ------------------------------------------------------------------ our arm

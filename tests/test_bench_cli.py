@@ -1,6 +1,7 @@
 """bench.py's command-line contract, on the CPU: the reference arm (the fp64 oracle timed
 on host cores) prints one JSON line with the contract's keys; under a multi-rank launch
-only rank 0 prints; fewer than 3 warm-up steps are refused."""
+only rank 0 prints; fewer than 3 warm-up steps are refused; the CPU baseline reports the
+oracle on all host cores and on one thread."""
 import json
 import os
 import subprocess
@@ -41,3 +42,18 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_too_few_warmup_steps_are_refused():
     r = _bench("--warmup", "2")
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    sys.path.insert(0, ROOT)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from mhc_hyper_connections_b200 import workloads as wl
+    w = wl.make_config("tiny_f32_T64_n4_d64")
+    cb = bench.cpu_baseline(w, seconds=0.2, chunk=16, single_seconds=0.1)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0 and cb["cores"] >= 1
+    one = cb["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and "one thread" in one["sample"]
+    json.dumps(cb)
