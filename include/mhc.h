@@ -1,5 +1,6 @@
 /*
- * mhc.h -- C ABI of the B200 (sm_100a) mHC forward hot path.
+ * mhc.h -- C ABI of the B200 (sm_100a) mHC layer: the pre and post stages, their
+ * backward, and the Amax gain diagnostic.
  *
  * mHC (Manifold-Constrained Hyper-Connections) keeps n residual streams per token,
  * X_t in R^{n x d}, and wraps every sub-layer F in two per-token stages:
@@ -20,8 +21,10 @@
  *
  * Conventions shared by every entry point
  *   - All data pointers are DEVICE pointers.  The caller allocates and owns every
- *     buffer; the library allocates no device memory and keeps no state between
- *     calls except a per-device cache of kernel launch limits.
+ *     buffer; the library allocates no device memory.  Between calls it keeps a
+ *     per-device cache of kernel launch limits and, in its device image, the status
+ *     word of the bounded waits (mhc_device_status) and the fixed scratch array of
+ *     mhc_backward_noalloc.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Arguments are validated on the host before any launch; a rejected
  *     call launches nothing and returns a non-zero mhc_status.  MHC_ERR_CUDA means
