@@ -1,4 +1,5 @@
-"""mhc_hyper_connections_b200 -- B200-native (sm_100a) mHC forward hot path.
+"""mhc_hyper_connections_b200 -- B200-native (sm_100a) mHC layer: pre and post stages, their
+backward, and the Amax gain diagnostic.
 
 Thin Python binding over the C ABI in include/mhc.h (libmhc_b200.so, built in-tree by
 ``python -m mhc_hyper_connections_b200.build``).  The functions here only marshal
@@ -12,6 +13,8 @@ CPU fallback -- if the library is missing the calls raise.
     mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
                  eps, t_max, H, h, dX_out, dx_in, dX, dF_out, dphi, db_pre, db_post,
                  db_res, dalpha, workspace)  -> the gradients of <dX_out, X'> + <dx_in, x_in>
+    mhc_backward_noalloc(...)       -> the same, in the library's fixed scratch array
+    mhc_amax_gain(H_layers, gain)   -> per-prefix row / column gains of H_res(l) ... H_res(1)
 
 Tensors are torch CUDA tensors (contiguous; X/F_out/x_in/X_out bf16 or fp32, phi, biases
 and H fp32).  Calls are asynchronous on the current torch stream unless ``stream`` (a
@@ -231,6 +234,29 @@ def mhc_backward_workspace_bytes(T: int, n: int, d: int) -> int:
     return int(load_library().mhc_backward_workspace_bytes(int(T), int(n), int(d)))
 
 
+def _backward_shapes(where, X, F_out, phi, b_pre, b_post, b_res, H, h, dX_out, dx_in, dX,
+                     dF_out, dphi, db_pre, db_post, db_res, dalpha):
+    """Check the shapes the backward reads and writes: the C ABI sees only pointers, so a
+    tensor smaller than its shape here would be read or written past its end."""
+    import torch
+    if X.dim() != 3:
+        raise ValueError(f"{where}: X must be [T, n, d]")
+    T, n, d = X.shape
+    m = n * n + 2 * n
+    full = (("F_out", F_out, (T, d)), ("dx_in", dx_in, (T, d)), ("dF_out", dF_out, (T, d)),
+            ("dX_out", dX_out, (T, n, d)), ("dX", dX, (T, n, d)), ("phi", phi, (n * d, m)),
+            ("dphi", dphi, (n * d, m)), ("H", H, (T, m)), ("h", h, (T, m)))
+    for name, t, shape in full:
+        if isinstance(t, torch.Tensor) and tuple(t.shape) != shape:
+            raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected {shape}")
+    counts = (("b_pre", b_pre, n), ("b_post", b_post, n), ("b_res", b_res, n * n),
+              ("db_pre", db_pre, n), ("db_post", db_post, n), ("db_res", db_res, n * n),
+              ("dalpha", dalpha, 3))
+    for name, t, cnt in counts:
+        if isinstance(t, torch.Tensor) and t.numel() != cnt:
+            raise ValueError(f"{where}: {name} needs {cnt} entries, has {t.numel()}")
+
+
 def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
                  H, h, dX_out, dx_in, dX, dF_out, dphi, db_pre, db_post, db_res, dalpha, workspace,
                  stream=None):
@@ -239,6 +265,8 @@ def mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alp
     db_res [n, n], dalpha [3] = (pre, post, res) fp32.  workspace: a CUDA tensor of at least
     mhc_backward_workspace_bytes(T, n, d) bytes."""
     import torch
+    _backward_shapes("mhc_backward", X, F_out, phi, b_pre, b_post, b_res, H, h, dX_out, dx_in, dX,
+                     dF_out, dphi, db_pre, db_post, db_res, dalpha)
     T, n, d = X.shape
     dev = X.device
     f32 = torch.float32
@@ -269,6 +297,8 @@ def mhc_backward_noalloc(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_p
     buffer.  Raises MhcError(MHC_ERR_WORKSPACE) for sizes that need more.  All calls on a
     device share that array, so calls that overlap on the GPU must be ordered."""
     import torch
+    _backward_shapes("mhc_backward_noalloc", X, F_out, phi, b_pre, b_post, b_res, H, h, dX_out,
+                     dx_in, dX, dF_out, dphi, db_pre, db_post, db_res, dalpha)
     T, n, d = X.shape
     dev = X.device
     f32 = torch.float32
