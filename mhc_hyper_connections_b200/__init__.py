@@ -159,15 +159,15 @@ def mhc_pre_with_path(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha
     T, n, d = X.shape
     dev = X.device
     f32 = torch.float32
-    ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
-                b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
-                b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
-                H=_ptr(H, "H", f32, dev))
     m = n * n + 2 * n
     if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m):
         raise ValueError("mhc_pre: shapes must be phi [n*d, m], x_in [T, d], H [T, m]")
     if b_pre.numel() != n or b_post.numel() != n or b_res.numel() != n * n:
         raise ValueError("mhc_pre: b_pre/b_post need n entries, b_res n*n")
+    ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
+                b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
+                b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
+                H=_ptr(H, "H", f32, dev))
     lib = load_library()
     with torch.cuda.device(dev):
         st = lib.mhc_pre_with_path(ptrs["X"], ptrs["phi"], ptrs["b_pre"], ptrs["b_post"],
@@ -192,13 +192,13 @@ def mhc_post(X, F_out, H, X_out, stream=None):
     import torch
     T, n, d = X.shape
     dev = X.device
+    if tuple(F_out.shape) != (T, d) or tuple(H.shape) != (T, n * n + 2 * n) or \
+            tuple(X_out.shape) != (T, n, d):
+        raise ValueError("mhc_post: shapes must be F_out [T, d], H [T, m], X_out [T, n, d]")
     px = _ptr(X, "X", device=dev)
     pf = _ptr(F_out, "F_out", X.dtype, dev)
     ph = _ptr(H, "H", torch.float32, dev)
     po = _ptr(X_out, "X_out", X.dtype, dev)
-    if tuple(F_out.shape) != (T, d) or tuple(H.shape) != (T, n * n + 2 * n) or \
-            tuple(X_out.shape) != (T, n, d):
-        raise ValueError("mhc_post: shapes must be F_out [T, d], H [T, m], X_out [T, n, d]")
     lib = load_library()
     with torch.cuda.device(dev):
         st = lib.mhc_post(px, pf, ph, T, n, d, _dt(X), po, _stream(stream, dev))
@@ -213,13 +213,15 @@ def mhc_pre_train(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res
     dev = X.device
     f32 = torch.float32
     m = n * n + 2 * n
+    if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m) \
+            or tuple(h.shape) != (T, m):
+        raise ValueError("mhc_pre_train: shapes must be phi [n*d, m], x_in [T, d], H and h [T, m]")
+    if b_pre.numel() != n or b_post.numel() != n or b_res.numel() != n * n:
+        raise ValueError("mhc_pre_train: b_pre/b_post need n entries, b_res n*n")
     ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
                 b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
                 b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
                 H=_ptr(H, "H", f32, dev), h=_ptr(h, "h", f32, dev))
-    if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m) \
-            or tuple(h.shape) != (T, m):
-        raise ValueError("mhc_pre_train: shapes must be phi [n*d, m], x_in [T, d], H and h [T, m]")
     lib = load_library()
     with torch.cuda.device(dev):
         st = lib.mhc_pre_train(ptrs["X"], ptrs["phi"], ptrs["b_pre"], ptrs["b_post"], ptrs["b_res"],

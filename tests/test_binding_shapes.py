@@ -1,4 +1,5 @@
-"""The binding's shape checks for mhc_backward and mhc_backward_noalloc, on the CPU.
+"""The binding's shape checks, on the CPU: mhc_backward and mhc_backward_noalloc, and the
+forward bindings mhc_pre, mhc_pre_train and mhc_post.
 
 The C ABI receives only pointers, so the binding checks every tensor's shape before a
 call: a tensor smaller than the backward expects would be read or written past its end.
@@ -8,7 +9,6 @@ earlier, naming the tensor.  The accepted cases build their tensors the way the 
 the benchmark and the smoke test do."""
 import dataclasses
 
-import numpy as np
 import pytest
 
 from mhc_hyper_connections_b200 import workloads as wl
@@ -121,3 +121,61 @@ def test_X_must_be_three_dimensional():
     a["X"] = a["X"].reshape(w.T, -1)
     with pytest.raises(ValueError, match=r"X must be \[T, n, d\]"):
         _call(a)
+
+
+def _fwd(w):
+    t = torch_inputs(w, device="cpu")
+    return (t, torch.empty(w.T, w.d, dtype=t["X"].dtype), torch.empty(w.T, w.m), torch.empty(w.T, w.m),
+            torch.empty_like(t["X"]))
+
+
+@pytest.mark.parametrize("w", CASES[:4] + [wl.make_inputs(T=9, n=8, d=16, dtype="bf16", seed=10)],
+                         ids=lambda w: w.name)
+def test_forward_shapes_of_the_gpu_tests_pass_the_check(w):
+    t, x_in, H, h, Y = _fwd(w)
+    sc = (0.01, 0.01, 0.01, 1e-20, 20)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        mhc.mhc_pre(t["X"], t["phi"], t["b_pre"], t["b_post"], t["b_res"], *sc, x_in, H)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        mhc.mhc_pre_train(t["X"], t["phi"], t["b_pre"], t["b_post"], t["b_res"], *sc, x_in, H, h)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        mhc.mhc_post(t["X"], t["F"], H, Y)
+
+
+@pytest.mark.parametrize("fn", ["mhc_pre", "mhc_pre_train"])
+@pytest.mark.parametrize("name,bad,msg", [
+    ("phi", lambda w: torch.empty(w.n * w.d, w.m + 1), "shapes must be"),
+    ("x_in", lambda w: torch.empty(w.T, w.d - 1, dtype=torch.bfloat16), "shapes must be"),
+    ("H", lambda w: torch.empty(w.T - 1, w.m), "shapes must be"),
+    ("b_pre", lambda w: torch.empty(w.n - 1), "need n entries"),
+    ("b_post", lambda w: torch.empty(w.n + 1), "need n entries"),
+    ("b_res", lambda w: torch.empty(w.n), "need n entries"),
+])
+def test_forward_wrong_shapes_are_refused(fn, name, bad, msg):
+    w = wl.make_inputs(T=16, n=4, d=64, dtype="bf16", seed=11)
+    t, x_in, H, h, _ = _fwd(w)
+    a = dict(X=t["X"], phi=t["phi"], b_pre=t["b_pre"], b_post=t["b_post"], b_res=t["b_res"], x_in=x_in, H=H)
+    a[name] = bad(w)
+    extra = (h,) if fn == "mhc_pre_train" else ()
+    with pytest.raises(ValueError, match=f"{fn}: .*{msg}"):
+        getattr(mhc, fn)(a["X"], a["phi"], a["b_pre"], a["b_post"], a["b_res"], 0.01, 0.01, 0.01, 1e-20, 20,
+                         a["x_in"], a["H"], *extra)
+
+
+def test_pre_train_checks_h():
+    w = wl.make_inputs(T=16, n=4, d=64, dtype="bf16", seed=12)
+    t, x_in, H, _, _ = _fwd(w)
+    with pytest.raises(ValueError, match="mhc_pre_train: shapes must be"):
+        mhc.mhc_pre_train(t["X"], t["phi"], t["b_pre"], t["b_post"], t["b_res"], 0.01, 0.01, 0.01, 1e-20, 20,
+                          x_in, H, torch.empty(w.T, w.m - 1))
+
+
+@pytest.mark.parametrize("name", ["F_out", "H", "X_out"])
+def test_post_wrong_shapes_are_refused(name):
+    w = wl.make_inputs(T=16, n=4, d=64, dtype="bf16", seed=13)
+    t, _, H, _, Y = _fwd(w)
+    a = dict(F_out=t["F"], H=H, X_out=Y)
+    a[name] = {"F_out": torch.empty(w.T, w.d + 8, dtype=torch.bfloat16), "H": torch.empty(w.T, w.m - 2),
+               "X_out": torch.empty(w.T, w.n - 1, w.d, dtype=torch.bfloat16)}[name]
+    with pytest.raises(ValueError, match="mhc_post: shapes must be"):
+        mhc.mhc_post(t["X"], a["F_out"], a["H"], a["X_out"])
