@@ -177,24 +177,25 @@ void oracle_mhc_projection(const double* X, const double* phi, long T, int n, in
 }
 
 /* Reverse mode through one token of pre + post (the chain rule applied to the forward
- * steps above, last step first).  Accumulates into the per-thread parameter gradients
- * gphi [nd*m], gb [m] (ordered [pre | res | post]) and ga [3] (pre, post, res: the order
- * of the alpha arguments).
- * work: [nd (x_hat) + nd (dx_hat) + m (h) + m (dl) + n*n*(2*t_max+1) (iterates) + 2*n*n]. */
+ * steps above, last step first).  Besides dX and dF_out of the token it returns what the
+ * token adds to the parameter gradients: dl [m], the gradient of the logits (ordered
+ * [pre | res | post], also the token's term of db), dh [m] = alpha dl, the gradient of the
+ * projection h, ga [3], the token's terms of dalpha (pre, post, res: the order of the
+ * alpha arguments), and its RMS r, so that its term of dphi is (X_t / r) dh^T.
+ * work: [nd (x_hat) + nd (dx_hat) + m (h) + n*n*(2*t_max+1) (iterates) + 2*n*n]. */
 static void backward_one_token(const double* Xt, const double* Ft, const double* phi,
                                const double* b_pre, const double* b_post, const double* b_res,
                                double alpha_pre, double alpha_post, double alpha_res,
                                int n, int d, double eps, int t_max,
                                const double* dYt, const double* dxt,
-                               double* dXt, double* dFt, double* gphi, double* gb, double* ga,
-                               double* work)
+                               double* dXt, double* dFt, double* dl, double* dh, double* ga,
+                               double* r_out, double* work)
 {
     const int nd = n * d, nn = n * n, m = nn + 2 * n;
     double* xhat = work;
     double* dxhat = xhat + nd;
     double* h = dxhat + nd;
-    double* dl = h + m;                   /* [dl_pre | dl_res | dl_post] */
-    double* it = dl + m;                  /* iterates M^(0..2 t_max), each n*n */
+    double* it = h + m;                   /* iterates M^(0..2 t_max), each n*n */
     double* gM = it + nn * (2 * t_max + 1);
     double* gA = gM + nn;
 
@@ -202,6 +203,7 @@ static void backward_one_token(const double* Xt, const double* Ft, const double*
     double ss = 0.0;
     for (int k = 0; k < nd; ++k) ss += Xt[k] * Xt[k];
     const double r = sqrt(ss / (double)nd + eps);
+    *r_out = r;
     for (int k = 0; k < nd; ++k) xhat[k] = Xt[k] / r;
     for (int j = 0; j < m; ++j) h[j] = 0.0;
     for (int k = 0; k < nd; ++k)
@@ -275,22 +277,18 @@ static void backward_one_token(const double* Xt, const double* Ft, const double*
         }
     }
     for (int q = 0; q < nn; ++q) dl[n + q] = gM[q] * it[q];      /* M0 = exp(l_res) */
-    /* ---- logits l = alpha h + b */
-    for (int j = 0; j < m; ++j) gb[j] += dl[j];
-    double dh[8 * 8 + 16];
+    /* ---- logits l = alpha h + b: db gets dl, dalpha gets <dl, h> per group */
+    ga[0] = ga[1] = ga[2] = 0.0;
     for (int i = 0; i < n; ++i) { ga[0] += dl[i] * h[i]; dh[i] = alpha_pre * dl[i]; }
     for (int q = 0; q < nn; ++q) { ga[2] += dl[n + q] * h[n + q]; dh[n + q] = alpha_res * dl[n + q]; }
     for (int i = 0; i < n; ++i) {
         ga[1] += dl[n + nn + i] * h[n + nn + i];
         dh[n + nn + i] = alpha_post * dl[n + nn + i];
     }
-    /* ---- projection h = x_hat phi */
+    /* ---- projection h = x_hat phi (dphi gets x_hat dh^T, summed by the caller) */
     for (int k = 0; k < nd; ++k) {
         double acc = 0.0;
-        for (int j = 0; j < m; ++j) {
-            gphi[(long)k * m + j] += xhat[k] * dh[j];
-            acc += phi[(long)k * m + j] * dh[j];
-        }
+        for (int j = 0; j < m; ++j) acc += phi[(long)k * m + j] * dh[j];
         dxhat[k] = acc;
     }
     /* ---- RMSNorm x_hat = v / r, r = sqrt(sum v^2 / nd + eps) */
@@ -311,21 +309,17 @@ void oracle_mhc_backward(const double* X, const double* F_out, const double* phi
 {
     const int nd = n * d, nn = n * n, m = nn + 2 * n;
     if (nthreads <= 0) nthreads = 1;
-    const size_t wlen = (size_t)(2 * nd + 2 * m + nn * (2 * t_max + 1) + 2 * nn);
-    const size_t plen = (size_t)nd * m + m + 3;          /* per-thread parameter sums */
-    double* part = (double*)calloc((size_t)nthreads * plen, sizeof(double));
+    const size_t wlen = (size_t)(2 * nd + m + nn * (2 * t_max + 1) + 2 * nn);
+    /* per-token terms of the parameter gradients */
+    double* dl = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * m);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * m);
+    double* ga = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * 3);
+    double* rt = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
 #ifdef _OPENMP
 #pragma omp parallel num_threads(nthreads)
 #endif
     {
-        int tid = 0;
-#ifdef _OPENMP
-        tid = omp_get_thread_num();
-#endif
         double* work = (double*)malloc(sizeof(double) * wlen);
-        double* gphi = part + (size_t)tid * plen;
-        double* gb = gphi + (size_t)nd * m;
-        double* ga = gb + m;
 #ifdef _OPENMP
 #pragma omp for schedule(static)
 #endif
@@ -333,28 +327,46 @@ void oracle_mhc_backward(const double* X, const double* F_out, const double* phi
             backward_one_token(X + t * (long)nd, F_out + t * (long)d, phi, b_pre, b_post, b_res,
                                alpha_pre, alpha_post, alpha_res, n, d, eps, t_max,
                                dX_out + t * (long)nd, dx_in + t * (long)d,
-                               dX + t * (long)nd, dF_out + t * (long)d, gphi, gb, ga, work);
+                               dX + t * (long)nd, dF_out + t * (long)d, dl + t * (long)m,
+                               dh + t * (long)m, ga + 3 * t, rt + t, work);
         free(work);
     }
-    /* thread partials summed in thread order */
-    for (size_t q = 0; q < (size_t)nd * m; ++q) {
-        double s = 0.0;
-        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + q];
-        dphi[q] = s;
+    /* The parameter gradients are sums over the tokens, each taken in token order:
+     * dphi[k][j] = sum_t (X_t[k] / r_t) dh_t[j], db = sum_t dl_t, dalpha = sum_t ga_t.
+     * Threads split the entries of dphi, never a sum, so the thread count does not
+     * change any result. */
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (long k0 = 0; k0 < nd; k0 += 8) {            /* 8 entries of a row of X per pass */
+        const int kb = (nd - k0) < 8 ? (int)(nd - k0) : 8;
+        double acc[8][8 * 8 + 16];
+        for (int u = 0; u < kb; ++u)
+            for (int j = 0; j < m; ++j) acc[u][j] = 0.0;
+        for (long t = 0; t < T; ++t)
+            for (int u = 0; u < kb; ++u) {
+                const double xh = X[t * (long)nd + k0 + u] / rt[t];
+                for (int j = 0; j < m; ++j) acc[u][j] += xh * dh[t * (long)m + j];
+            }
+        for (int u = 0; u < kb; ++u)
+            for (int j = 0; j < m; ++j) dphi[(k0 + u) * (long)m + j] = acc[u][j];
     }
     for (int j = 0; j < m; ++j) {
         double s = 0.0;
-        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + (size_t)nd * m + j];
+        for (long t = 0; t < T; ++t) s += dl[t * (long)m + j];
         if (j < n) db_pre[j] = s;
         else if (j < n + nn) db_res[j - n] = s;
         else db_post[j - n - nn] = s;
     }
     for (int a = 0; a < 3; ++a) {
         double s = 0.0;
-        for (int p = 0; p < nthreads; ++p) s += part[(size_t)p * plen + (size_t)nd * m + m + a];
+        for (long t = 0; t < T; ++t) s += ga[3 * t + a];
         dalpha[a] = s;
     }
-    free(part);
+    free(dl);
+    free(dh);
+    free(ga);
+    free(rt);
 }
 
 /* Amax Gain Magnitude of the composite residual maps ("DeepSeek-V4/mhc" page, the

@@ -66,7 +66,8 @@ void oracle_mhc_projection(const double* X, const double* phi, long T, int n, in
  * scratch.  Outputs: dX [T, n, d] (through the projection, RMSNorm, the read map and the
  * merge), dF_out [T, d], dphi [n*d, m], db_pre [n], db_post [n], db_res [n*n] and
  * dalpha [3] = (pre, post, res) -- the order of the alpha arguments -- the parameter
- * gradients summed over all T tokens. */
+ * gradients summed over all T tokens, each sum taken in token order (threads split the
+ * tokens' own terms and the entries of dphi, never a sum). */
 void oracle_mhc_backward(const double* X, const double* F_out, const double* phi,
                          const double* b_pre, const double* b_post, const double* b_res,
                          double alpha_pre, double alpha_post, double alpha_res,

@@ -124,3 +124,21 @@ def test_projection_is_scale_invariant_and_feeds_the_gates():
     _, H = oracle.mhc_pre(p["X"], p["phi"], p["b_pre"], p["b_post"], p["b_res"], *p["alpha"])
     Hp = 1.0 / (1.0 + np.exp(-(p["alpha"][0] * h[:, :4] + p["b_pre"])))
     assert np.allclose(H[:, :4], Hp, rtol=1e-14, atol=1e-15)
+
+
+def test_parameter_gradients_are_token_sums_independent_of_threads():
+    """dphi, db and dalpha are sums over tokens: the oracle over all tokens equals, bit for
+    bit, itself on 1, 3 and 8 threads, and agrees with the sum of per-token oracle calls."""
+    p = _problem(37, 3, 5, seed=12)
+    s = dict(eps=1e-20, t_max=20)
+
+    def run(X, F, dY, dx, k):
+        return oracle.mhc_backward(X, F, p["phi"], p["b_pre"], p["b_post"], p["b_res"], *p["alpha"],
+                                   dY, dx, nthreads=k, **s)
+    runs = [run(p["X"], p["F"], p["dY"], p["dx"], k) for k in (1, 3, 8)]
+    for k in runs[0]:
+        assert all(np.array_equal(runs[0][k], r[k]) for r in runs[1:]), k
+    per_token = [run(p["X"][t:t + 1], p["F"][t:t + 1], p["dY"][t:t + 1], p["dx"][t:t + 1], 1) for t in range(37)]
+    for k in ("dphi", "db_pre", "db_post", "db_res", "dalpha"):
+        total = sum(g[k] for g in per_token)
+        assert np.allclose(runs[0][k], total, rtol=1e-12, atol=1e-14 * np.abs(total).max()), k
