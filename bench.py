@@ -7,9 +7,10 @@
 One step = mhc_pre + mhc_post over one batch of T tokens (the whole hot path; F_out is a
 given input, the sub-layer F itself is not part of the path).  Default workload: T = 16384
 tokens (4 x 4096), n = 4 streams, d = 4096, bf16 storage, fp32 arithmetic, 1 % outlier
-channels; inputs are synthetic and seeded (mhc_hyper_connections_b200.workloads).  The
-workload's inputs (X 512 MiB + F_out 128 MiB) are larger than L2, so no L2 flush is
-needed between steps.
+channels; inputs are synthetic and seeded (mhc_hyper_connections_b200.workloads).  A step's
+buffers at that size (X 512 MiB + F_out 128 MiB + outputs) are far larger than L2, so no
+flush is needed between steps; for a workload whose buffers are smaller than twice the L2,
+the timed loop rotates through enough copies of them to cover three times the L2.
 
 Multi-GPU: tokens are independent, so every rank runs its own T-token batch (weak
 scaling, no data-path collective); the time is the max over ranks.
@@ -76,6 +77,39 @@ def bytes_per_token(n, d, es):
     pre = (n + 1) * d * es + 4 * m
     post = (2 * n + 1) * d * es + 4 * (n * n + n)
     return pre, post
+
+
+L2_BYTES = 126 * 2 ** 20           # B200 L2 (the device's own figure is used when known)
+
+
+def buffer_sets(T, n, d, es, l2_bytes=L2_BYTES):
+    """How many copies of the step's buffers (X, F_out, x_in, H, X') the timed loop rotates
+    through so that no step finds the previous step's data in L2: one when a single set is
+    at least twice the L2, else enough sets to cover three times the L2 (at least four, at
+    most 64: a step that small is bound by its launches, not by memory)."""
+    m = n * n + 2 * n
+    one = T * (2 * n + 2) * d * es + T * m * 4
+    if one >= 2 * l2_bytes:
+        return 1, one
+    return min(64, max(4, -(-3 * l2_bytes // one))), one
+
+
+def workload_config(w, world, l2_bytes=L2_BYTES):
+    """The `config` object of the JSON line, the same for both arms: what the workload is,
+    not how an arm ran it."""
+    es = 2 if w.dtype == "bf16" else 4
+    sets, one = buffer_sets(w.T, w.n, w.d, es, l2_bytes)
+    mib = lambda b: f"{b / 2 ** 20:.0f} MiB" if b >= 2 ** 20 else f"{b / 2 ** 10:.0f} KiB"
+    if sets == 1:
+        l2 = (f"inputs larger than L2 (X {mib(w.T * w.n * w.d * es)} + F_out {mib(w.T * w.d * es)}; "
+              f"one step's buffers {mib(one)} vs L2 {mib(l2_bytes)}), no flush")
+    else:
+        l2 = (f"{sets} buffer sets of {mib(one)} rotated between steps ({mib(sets * one)} vs L2 "
+              f"{mib(l2_bytes)}), no flush")
+    s = w.scalars()
+    return {"workload": w.name.split("[")[0], "T": w.T, "n": w.n, "d": w.d, "storage": w.dtype,
+            "tokens_per_gpu": w.T, "parallelism": f"replicas x{world} (token shards, no collective)",
+            "l2": l2, "alpha": s["alpha_pre"], "t_max": s["t_max"], "eps": s["eps"]}
 
 
 # ------------------------------------------------------------------ clocks
@@ -182,8 +216,7 @@ def run_reference(args, rank, world):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.config, "T": w.T, "n": w.n, "d": w.d,
-                   "storage": w.dtype, "tokens_per_step": per_step},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
                          "sample": f"{per_step} random tokens of the {w.T}-token batch per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -274,26 +307,36 @@ def run_ours(args, rank, world, local_rank):
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
-    X, F = to_dev(w.X), to_dev(w.F_out)
+    l2_bytes = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or L2_BYTES
+    nsets, _ = buffer_sets(T, n, d, es, l2_bytes)
+    X0, F0 = to_dev(w.X), to_dev(w.F_out)
     phi, b_pre, b_post, b_res = (to_dev(a) for a in (w.phi, w.b_pre, w.b_post, w.b_res))
-    x_in = torch.empty(T, d, dtype=tdt, device=dev)
-    H = torch.empty(T, w.m, dtype=torch.float32, device=dev)
-    Y = torch.empty_like(X)
+    # nsets copies of the step's buffers, rotated so that no step reads the previous step's
+    # data out of L2 (one set when a set is at least twice the L2)
+    bufs = []
+    for i in range(nsets):
+        Xi, Fi = (X0, F0) if i == 0 else (X0.clone(), F0.clone())
+        bufs.append(dict(X=Xi, F=Fi, x_in=torch.empty(T, d, dtype=tdt, device=dev),
+                         H=torch.empty(T, w.m, dtype=torch.float32, device=dev),
+                         Y=torch.empty_like(Xi)))
+    X, F, x_in, H, Y = (bufs[0][k] for k in ("X", "F", "x_in", "H", "Y"))
     s = w.scalars()
     req = {"auto": mhc.PRE_AUTO, "generic": mhc.PRE_GENERIC,
            "cluster_tc": mhc.PRE_CLUSTER_TC}[args.pre_path]
     path = mhc.mhc_pre_path_for(T, n, d, tdt) if req == mhc.PRE_AUTO else req
 
-    def pre():
-        mhc.mhc_pre_with_path(X, phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
-                              s["alpha_res"], s["eps"], s["t_max"], x_in, H, path=req)
+    def pre(k=0):
+        b = bufs[k % nsets]
+        mhc.mhc_pre_with_path(b["X"], phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
+                              s["alpha_res"], s["eps"], s["t_max"], b["x_in"], b["H"], path=req)
 
-    def post():
-        mhc.mhc_post(X, F, H, Y)
+    def post(k=0):
+        b = bufs[k % nsets]
+        mhc.mhc_post(b["X"], b["F"], b["H"], b["Y"])
 
-    for _ in range(args.warmup):
-        pre()
-        post()
+    for k in range(args.warmup):
+        pre(k)
+        post(k)
     torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps, events on the launching (current) stream
@@ -310,9 +353,9 @@ def run_ours(args, rank, world, local_rank):
     for k in range(K):
         e = evs[k]
         e[0].record()
-        pre()
+        pre(k)
         e[1].record()
-        post()
+        post(k)
         e[2].record()
     end.record()
     torch.cuda.synchronize()
@@ -402,10 +445,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_total / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": {"workload": args.config, "T": T, "n": n, "d": d, "tokens_per_gpu": T,
-                   "parallelism": f"replicas x{world} (token shards, no collective)",
-                   "l2": "inputs larger than L2 (X 512 MiB + F_out 128 MiB), no flush",
-                   "alpha": s["alpha_pre"], "t_max": s["t_max"], "eps": s["eps"]},
+        "config": workload_config(w, world, l2_bytes),
         "roofline": roofline, "hbm": hbm, "kernels": kern, "clocks": clocks, "e2e": e2e,
         "cpu_baseline": cpu, "gpu_launches": 2 * K,
     }

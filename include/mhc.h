@@ -193,16 +193,21 @@ mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, cons
  * a cudaMalloc (which can synchronise the device) is not allowed.  The paper has no
  * counterpart to this; it is a library convenience.
  *
- * Same arguments, results and errors as mhc_backward, minus the workspace pair.  The
- * workspace is a fixed array of MHC_NOALLOC_SCRATCH_BYTES bytes inside the library's device
- * image: every device on which the library's code is loaded holds it until the process
- * exits, and the call itself allocates nothing (no cudaMalloc, no cudaFree).
+ * Same arguments, results and errors as mhc_backward, minus the workspace pair, and checked
+ * in the same order.  The workspace is a fixed array of MHC_NOALLOC_SCRATCH_BYTES bytes
+ * inside the library's device image: every device on which the library's code is loaded
+ * holds it until the process exits, and the call itself allocates nothing (no cudaMalloc,
+ * no cudaFree).
  *   - Sizes whose mhc_backward_workspace_bytes(T, n, d) exceeds MHC_NOALLOC_SCRATCH_BYTES
- *     are rejected with MHC_ERR_WORKSPACE, launching nothing (T = 16384, n = 4, d = 4096
- *     needs 30.0 MB and fits).
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current) and caches it; make that first call before any stream
- *     capture on the device.
+ *     fail mhc_backward's workspace check: MHC_ERR_WORKSPACE, after the pointer, shape and
+ *     alignment checks, launching nothing (T = 16384, n = 4, d = 4096 needs 30.0 MB and
+ *     fits).
+ *   - The first call on a device (T > 0) looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it for the device's
+ *     current CUDA context; a later context on the device (after cudaDeviceReset, say)
+ *     gets a new lookup.  Make the first call on each device, and the first after a reset,
+ *     before any stream capture on it.  If the lookup fails the call returns MHC_ERR_CUDA
+ *     before any other check.
  *   - All calls on a device share the one array, which keeps whatever the last call left
  *     in it.  Nothing in it needs to start at zero (every kernel writes its part before
  *     reading it), but calls that overlap on the GPU -- on different streams, or from

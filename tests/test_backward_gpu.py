@@ -162,6 +162,30 @@ def test_headline_size_sampled_and_additive():
     assert all(np.isfinite(full[k]).all() for k in GRADS)
 
 
+def test_headline_size_all_tokens():
+    """The forward-plus-backward workload at full size (T=16384, n=4, d=4096, bf16 with
+    outlier channels): the parameter gradients, summed on the GPU over all 16384 tokens,
+    against the oracle's sums over all tokens (run in token chunks, the chunk sums added in
+    token order); dX and dF_out on 1056 tokens (the first 16, the last 16 and 1024 drawn)."""
+    import os
+    w = wl.make_config(wl.HEADLINE)
+    dY, dx = _upstream(w, 105)
+    rng = np.random.default_rng(9)
+    rows = np.unique(np.concatenate([np.arange(16), np.arange(w.T - 16, w.T),
+                                     rng.choice(np.arange(16, w.T - 16), 1024, replace=False)]))
+    full = run_gpu(w, dY, dx, rows=rows)
+    cores = os.cpu_count() or 8
+    params = ("dphi", "db_pre", "db_post", "db_res", "dalpha")
+    ref = {k: 0.0 for k in params}
+    for c0 in range(0, w.T, 2048):
+        part = run_oracle(w, dY, dx, tokens=np.arange(c0, min(w.T, c0 + 2048)), nthreads=cores)
+        for k in params:
+            ref[k] = ref[k] + part[k]
+    check(w, full, ref, "headline all tokens", names=params)
+    check(w.tokens(rows), full, run_oracle(w, dY, dx, tokens=rows, nthreads=cores),
+          "headline 1056 tokens", names=("dX", "dF_out"))
+
+
 def test_saved_projection_matches_oracle_on_both_paths():
     for name in ("tiny_f32_T64_n4_d64", "bf16_T4096_n4_d1024"):
         w = wl.make_config(name)
