@@ -82,7 +82,8 @@ typedef enum {
     MHC_PRE_AUTO = 0,          /* the fastest path that supports the problem          */
     MHC_PRE_GENERIC = 1,       /* CUDA-core kernel: any n <= 8, any d, f32 or bf16    */
     MHC_PRE_CLUSTER_TC = 2     /* thread-block-cluster tensor-core kernel (bf16,      */
-                               /* n <= 4, d in {1024, 2048, 3072, 4096}; sm_100)      */
+                               /* n <= 4, d % 64 == 0, n*d >= 1024, phi slice fits    */
+                               /* shared memory, e.g. d <= 6144 at n = 4; sm_100)     */
 } mhc_pre_path;
 
 /*
@@ -248,6 +249,20 @@ mhc_status mhc_amax_gain(const float* H_layers, int L, int64_t T, int n, float* 
  * pages: this is the library's failure report.
  */
 mhc_status mhc_device_status(uint32_t* code);
+
+/*
+ * mhc_debug_pre_stop_after -- test hook for the failure path of the tensor-core pre kernel
+ * (MHC_PRE_CLUSTER_TC).  After this call, its launches stop loading X after `tiles` token
+ * tiles per cluster (tiles < 0: never, the default) and give up a wait after
+ * `wait_limit_us` microseconds (default 1000000; accepted range 1000 .. 10000000, else
+ * MHC_ERR_SHAPE).  Every cluster stops at the same tile boundary, so all the tiles before
+ * it complete; the waits that depend on the tiles never loaded run into their limit, the
+ * kernel sets bits in mhc_device_status, drains its own copies in flight (those drain
+ * waits keep a limit of at least 1 s) and returns with x_in and H incomplete.  The setting
+ * is process-wide and applies from the next launch.  No counterpart on the pages: a
+ * library test facility for the bounded waits.
+ */
+mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us);
 
 /* Static English text for a status code (never NULL). */
 const char* mhc_status_string(mhc_status status);

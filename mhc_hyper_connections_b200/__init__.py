@@ -28,7 +28,7 @@ import threading
 
 __all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_post", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
-           "mhc_amax_gain", "mhc_pre_path_for", "mhc_device_status",
+           "mhc_amax_gain", "mhc_pre_path_for", "mhc_device_status", "mhc_debug_pre_stop_after",
            "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
@@ -47,7 +47,7 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
 EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
                     "mhc_amax_gain", "mhc_status_string",
-                    "mhc_last_error", "mhc_device_status")
+                    "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after")
 
 _lock = threading.Lock()
 _lib = None
@@ -102,6 +102,8 @@ def load_library():
         lib.mhc_last_error.restype = ctypes.c_char_p
         lib.mhc_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         lib.mhc_device_status.restype = ci
+        lib.mhc_debug_pre_stop_after.argtypes = [ctypes.c_int32, ctypes.c_uint32]
+        lib.mhc_debug_pre_stop_after.restype = ci
         _lib = lib
     return _lib
 
@@ -346,6 +348,15 @@ def mhc_device_status() -> int:
     code = ctypes.c_uint32(0)
     _check(load_library().mhc_device_status(ctypes.byref(code)), "mhc_device_status")
     return int(code.value)
+
+
+def mhc_debug_pre_stop_after(tiles: int, wait_limit_us: int = 1_000_000) -> None:
+    """Test hook of the tensor-core pre kernel's failure path: later launches stop loading
+    after `tiles` token tiles per cluster (tiles < 0 restores normal operation) and give up
+    a wait after `wait_limit_us` microseconds.  The waits that depend on the tiles never
+    loaded expire, the kernel returns early and mhc_device_status() reports it."""
+    _check(load_library().mhc_debug_pre_stop_after(int(tiles), int(wait_limit_us)),
+           "mhc_debug_pre_stop_after")
 
 
 def mhc_pre_path_for(T: int, n: int, d: int, dtype) -> int:

@@ -48,13 +48,17 @@ cudaError_t device_info(DeviceInfo* out);
 
 cudaError_t launch_pre_generic(const PreArgs& a);
 
-// Cluster tensor-core path: shape test (host only) and launch.
-bool pre_cluster_tc_shape_ok(int64_t T, int n, int d, DType dt);
-// Whether the current device can run it for (n, d) (sm_100 and a resident 16-CTA cluster).
-bool pre_cluster_tc_device_ok(int n, int d);
-cudaError_t launch_pre_cluster_tc(const PreArgs& a);
-// Status word of the cluster kernel's bounded waits (0 = fine); optionally cleared.
-cudaError_t pre_cluster_tc_status(unsigned* out, bool clear);
+// Tensor-core path (16-CTA clusters): shape test (host only) and launch.
+bool pre_tc_shape_ok(int64_t T, int n, int d, DType dt);
+// Whether the current device can run it for (n, d) (sm_100, phi slice fits shared memory,
+// a resident 16-CTA cluster).
+bool pre_tc_device_ok(int n, int d);
+cudaError_t launch_pre_tc(const PreArgs& a);
+// Status word of the tensor-core kernel's bounded waits (0 = fine); optionally cleared.
+cudaError_t pre_tc_status(unsigned* out, bool clear);
+// Failure-path test hook: launches after this call stop loading after `stop_tile` tiles
+// per cluster (< 0: never) and give up a wait after `wait_ns`.
+void pre_tc_set_stop(int stop_tile, unsigned long long wait_ns);
 
 cudaError_t launch_post(const PostArgs& a);
 

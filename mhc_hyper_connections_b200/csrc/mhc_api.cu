@@ -118,7 +118,7 @@ extern "C" {
 mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
     if (check_shape(T, n, d, dt) != MHC_OK) return MHC_PRE_GENERIC;
     const DType t = dt == MHC_BF16 ? BF16 : F32;
-    if (pre_cluster_tc_shape_ok(T, n, d, t) && pre_cluster_tc_device_ok(n, d)) return MHC_PRE_CLUSTER_TC;
+    if (pre_tc_shape_ok(T, n, d, t) && pre_tc_device_ok(n, d)) return MHC_PRE_CLUSTER_TC;
     return MHC_PRE_GENERIC;
 }
 
@@ -137,11 +137,11 @@ static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, 
     a.h_out = h_out;
     cudaError_t e;
     if (path == MHC_PRE_CLUSTER_TC) {
-        if (!pre_cluster_tc_shape_ok(T, n, d, a.dt) || !pre_cluster_tc_device_ok(n, d))
+        if (!pre_tc_shape_ok(T, n, d, a.dt) || !pre_tc_device_ok(n, d))
             return MHC_ERR_UNSUPPORTED;
         if (!aligned(X, 16) || !aligned(x_in, 16) || !aligned(phi, 16)) return MHC_ERR_UNSUPPORTED;
-        e = launch_pre_cluster_tc(a);
-        if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (cluster tensor-core kernel)");
+        e = launch_pre_tc(a);
+        if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (tensor-core kernel)");
     } else {
         e = launch_pre_generic(a);
         if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (generic kernel)");
@@ -308,10 +308,16 @@ const char* mhc_status_string(mhc_status s) {
 
 const char* mhc_last_error(void) { return g_last_error; }
 
+mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us) {
+    if (wait_limit_us < 1000u || wait_limit_us > 10000000u) return MHC_ERR_SHAPE;
+    pre_tc_set_stop(tiles < 0 ? -1 : (int)tiles, (unsigned long long)wait_limit_us * 1000ull);
+    return MHC_OK;
+}
+
 mhc_status mhc_device_status(uint32_t* code) {
     if (!code) return MHC_ERR_NULL;
     unsigned v = 0;
-    cudaError_t e = pre_cluster_tc_status(&v, true);
+    cudaError_t e = pre_tc_status(&v, true);
     if (e != cudaSuccess) return cuda_fail(e, "mhc_device_status");
     *code = v;
     return MHC_OK;

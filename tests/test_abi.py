@@ -144,3 +144,11 @@ def test_amax_gain_validation(lib):
     assert lib.mhc_amax_gain(0, 3, 5, 4, A + 0x1000000, None) == 1
     assert lib.mhc_amax_gain(A, 3, 5, 4, A + 2, None) == 3
     assert lib.mhc_amax_gain(A, 3, 5, 4, A + 64, None) == 7             # gain overlaps H_layers
+
+
+def test_debug_stop_hook_validation(lib):
+    """The failure-path test hook checks its wait limit on the host; the default setting
+    (never stop, 1 s waits) is restored at the end."""
+    assert lib.mhc_debug_pre_stop_after(-1, 999) == 2
+    assert lib.mhc_debug_pre_stop_after(3, 10_000_001) == 2
+    assert lib.mhc_debug_pre_stop_after(-1, 1_000_000) == 0

@@ -103,6 +103,9 @@ SHAPES = [  # (T, n, d, dtype): ragged token tails, odd d, every n
     (19, 3, 40, "f32"), (7, 5, 24, "bf16"), (9, 8, 64, "f32"), (3, 4, 37, "bf16"),
     (100, 4, 2048, "bf16"), (50, 4, 3072, "bf16"), (31, 6, 16, "bf16"), (12, 7, 9, "f32"),
     (130, 4, 4096, "bf16"), (23, 2, 1024, "bf16"), (40, 1, 1024, "bf16"),
+    # tensor-core path at channel counts off the powers of two, several tiles per cluster
+    (77, 4, 2560, "bf16"), (65, 4, 5120, "bf16"), (1363, 4, 512, "bf16"), (200, 3, 1280, "bf16"),
+    (129, 2, 768, "bf16"), (1000, 1, 1024, "bf16"), (64 * 7 * 3 + 17, 4, 1024, "bf16"),
 ]
 
 
@@ -204,17 +207,20 @@ def test_paths_agree_with_each_other():
 
 
 def test_auto_path_on_b200_shapes_is_tensor_core():
-    """On a B200 the bf16 shapes with n <= 4 and d in {1024..4096} run the cluster
-    tensor-core kernel; everything else runs the generic kernel."""
+    """On a B200 the bf16 shapes with n <= 4, d a multiple of 64, n*d >= 1024 and a phi slice
+    that fits shared memory run the cluster tensor-core kernel; everything else runs the
+    generic kernel."""
     major, minor = torch.cuda.get_device_capability()
     if (major, minor) != (10, 0):
         pytest.skip("not an sm_100 device")
     for n in (1, 2, 3, 4):
-        for d in (1024, 2048, 3072, 4096):
+        for d in (1024, 2048, 2560, 3072, 4096, 5120):
             assert mhc.mhc_pre_path_for(16384, n, d, 1) == mhc.PRE_CLUSTER_TC, (n, d)
-    assert mhc.mhc_pre_path_for(16384, 4, 4096, 0) == mhc.PRE_GENERIC     # fp32 storage
-    assert mhc.mhc_pre_path_for(16384, 8, 4096, 1) == mhc.PRE_GENERIC     # n = 8
-    assert mhc.mhc_pre_path_for(16384, 4, 512, 1) == mhc.PRE_GENERIC      # d < 1024
+    assert mhc.mhc_pre_path_for(16384, 4, 512, 1) == mhc.PRE_CLUSTER_TC       # n*d = 2048
+    assert mhc.mhc_pre_path_for(16384, 4, 4096, 0) == mhc.PRE_GENERIC         # fp32 storage
+    assert mhc.mhc_pre_path_for(16384, 8, 4096, 1) == mhc.PRE_GENERIC         # n = 8
+    assert mhc.mhc_pre_path_for(16384, 4, 4100, 1) == mhc.PRE_GENERIC         # d % 64 != 0
+    assert mhc.mhc_pre_path_for(16384, 2, 256, 1) == mhc.PRE_GENERIC          # n*d < 1024
 
 
 def test_device_status_clean_after_runs():
@@ -236,9 +242,9 @@ def test_tensor_core_path_rejects_what_it_cannot_run():
 
 
 def test_single_atom_tiles_after_dirty_tmem():
-    """n = 1, d = 1024 gives one K atom per tile, so all but one of the tensor-core kernel's
+    """n = 1, d = 1024 gives one K atom per CTA, so all but one of the tensor-core kernel's
     MMA accumulators receive no MMA; they must not be added in.  A launch at n = 4 first
-    leaves non-zero accumulators and stashed X in TMEM on the same SMs."""
+    leaves non-zero accumulators in TMEM on the same SMs."""
     dirty = wl.make_inputs(T=2048, n=4, d=4096, dtype="bf16", seed=41)
     w = wl.make_inputs(T=300, n=1, d=1024, dtype="bf16", seed=42)
     ref = run_oracle(w)
