@@ -9,6 +9,9 @@ What each function follows (page title, section / equation):
                  slavadubrov.com mHC article, section "Sinkhorn-Knopp-projectie".
   * mhc_pre   -- "DeepSeek-V4/mhc" page, "动态参数化怎么实现": equations rmsnorm,
                  a/b/c-tilde and gate; slavadubrov.com article Eq. 3 (read map).
+  * hc_pre    -- the HC maps mHC is compared with: slavadubrov.com article,
+                 "Kernmechanismen" (a bias plus an input-dependent term through tanh)
+                 and "Details van de parameterisatie" (tanh is what mHC replaces).
   * mhc_post  -- slavadubrov.com article, "Kernmechanismen" Eq. 3; the knowledge
                  page's HC update equation.
   * mhc_projection -- the normalised projection h of the same page's rmsnorm and
@@ -63,6 +66,11 @@ def _load():
                                            ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_double, ctypes.c_int, _dp, _dp, ctypes.c_int]
             lib.oracle_mhc_pre.restype = None
+            lib.oracle_hc_pre.argtypes = [_dp, _dp, _dp, _dp, _dp,
+                                          ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                          ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_double, _dp, _dp, ctypes.c_int]
+            lib.oracle_hc_pre.restype = None
             lib.oracle_mhc_post.argtypes = [_dp, _dp, _dp, ctypes.c_long, ctypes.c_int,
                                             ctypes.c_int, _dp, ctypes.c_int]
             lib.oracle_mhc_post.restype = None
@@ -114,6 +122,24 @@ def mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
     _load().oracle_mhc_pre(_p(X), _p(phi), _p(b_pre), _p(b_post), _p(b_res),
                            float(alpha_pre), float(alpha_post), float(alpha_res),
                            T, n, d, float(eps), int(t_max), _p(x_in), _p(H), int(nthreads))
+    return x_in, H
+
+
+def hc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+           eps: float = 1e-20, nthreads: int = 1):
+    """HC pre stage (unconstrained maps: bias + alpha tanh(h), no Sinkhorn).
+    X [T, n, d] -> (x_in [T, d], H [T, n*n+2n]) in fp64."""
+    X = _c(X)
+    T, n, d = X.shape
+    m = n * n + 2 * n
+    phi = _c(phi)
+    assert phi.shape == (n * d, m), phi.shape
+    b_pre, b_post, b_res = _c(b_pre).reshape(n), _c(b_post).reshape(n), _c(b_res).reshape(n * n)
+    x_in = np.empty((T, d), np.float64)
+    H = np.empty((T, m), np.float64)
+    _load().oracle_hc_pre(_p(X), _p(phi), _p(b_pre), _p(b_post), _p(b_res),
+                          float(alpha_pre), float(alpha_post), float(alpha_res),
+                          T, n, d, float(eps), _p(x_in), _p(H), int(nthreads))
     return x_in, H
 
 

@@ -85,6 +85,69 @@ static void pre_one_token(const double* Xt, const double* phi,
     }
 }
 
+/* One token of the HC pre stage, the unconstrained comparison the mHC pages start from
+ * (slavadubrov.com article, section "Kernmechanismen": in HC each map is a learned static
+ * part, a bias, plus an input-dependent term passed through tanh, so its entries may take
+ * either sign; the same article's "Details van de parameterisatie" names tanh as what mHC
+ * replaces by the sigmoid).  The input-dependent term is read as the same normalised
+ * projection h = RMSNorm(vec X) . phi that mHC uses, scaled by the map's alpha:
+ *   H_pre = b_pre + alpha_pre tanh(h_pre), H_res = b_res + alpha_res tanh(Mat(h_res)),
+ *   H_post = b_post + alpha_post tanh(h_post)   (no exp, no Sinkhorn, no sigmoid);
+ * the read map is the same: x_in = sum_i H_pre[i] X[i, :].  work: [n*d + m] doubles. */
+static void hc_pre_one_token(const double* Xt, const double* phi,
+                             const double* b_pre, const double* b_post, const double* b_res,
+                             double alpha_pre, double alpha_post, double alpha_res,
+                             int n, int d, double eps, double* x_in_t, double* H_t, double* work)
+{
+    const int nd = n * d;
+    const int m = n * n + 2 * n;
+    double* xhat = work;          /* [nd] */
+    double* h = xhat + nd;        /* [m]  */
+
+    double ss = 0.0;
+    for (int k = 0; k < nd; ++k) ss += Xt[k] * Xt[k];
+    const double r = sqrt(ss / (double)nd + eps);
+    for (int k = 0; k < nd; ++k) xhat[k] = Xt[k] / r;
+    for (int j = 0; j < m; ++j) h[j] = 0.0;
+    for (int k = 0; k < nd; ++k)
+        for (int j = 0; j < m; ++j) h[j] += xhat[k] * phi[(long)k * m + j];
+
+    for (int i = 0; i < n; ++i) H_t[i] = b_pre[i] + alpha_pre * tanh(h[i]);
+    for (int k = 0; k < n * n; ++k) H_t[n + k] = b_res[k] + alpha_res * tanh(h[n + k]);
+    for (int i = 0; i < n; ++i)
+        H_t[n + n * n + i] = b_post[i] + alpha_post * tanh(h[n + n * n + i]);
+
+    for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += H_t[i] * Xt[i * d + c];
+        x_in_t[c] = acc;
+    }
+}
+
+void oracle_hc_pre(const double* X, const double* phi,
+                   const double* b_pre, const double* b_post, const double* b_res,
+                   double alpha_pre, double alpha_post, double alpha_res,
+                   long T, int n, int d, double eps, double* x_in, double* H, int nthreads)
+{
+    const int nd = n * d;
+    const int m = n * n + 2 * n;
+    if (nthreads <= 0) nthreads = 1;
+#ifdef _OPENMP
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double* work = (double*)malloc(sizeof(double) * (size_t)(nd + m));
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
+        for (long t = 0; t < T; ++t)
+            hc_pre_one_token(X + t * (long)nd, phi, b_pre, b_post, b_res,
+                             alpha_pre, alpha_post, alpha_res, n, d, eps,
+                             x_in + t * (long)d, H + t * (long)m, work);
+        free(work);
+    }
+}
+
 int oracle_threads_used(int nthreads)
 {
 #ifdef _OPENMP

@@ -50,6 +50,15 @@ void oracle_mhc_pre(const double* X, const double* phi,
                     long T, int n, int d, double eps, int t_max,
                     double* x_in, double* H, int nthreads);
 
+/* HC pre stage (the unconstrained maps mHC is compared with) over T tokens: the same
+ * RMSNorm and projection h, then H_pre = b_pre + alpha_pre tanh(h_pre),
+ * H_res = b_res + alpha_res tanh(Mat(h_res)), H_post = b_post + alpha_post tanh(h_post),
+ * and x_in = H_pre X.  Same layouts as oracle_mhc_pre; the post stage is oracle_mhc_post. */
+void oracle_hc_pre(const double* X, const double* phi,
+                   const double* b_pre, const double* b_post, const double* b_res,
+                   double alpha_pre, double alpha_post, double alpha_res,
+                   long T, int n, int d, double eps, double* x_in, double* H, int nthreads);
+
 /* Post stage over T tokens: X_out[t,i,c] = sum_j H_res[i][j] X[t,j,c] + H_post[i] F_out[t,c].
  * X [T, n, d]; F_out [T, d]; H [T, m] as written by oracle_mhc_pre; X_out [T, n, d]. */
 void oracle_mhc_post(const double* X, const double* F_out, const double* H,
