@@ -119,6 +119,25 @@ mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre
                              mhc_stream_t stream, mhc_pre_path path);
 
 /*
+ * mhc_pre_hc -- the pre stage with the HC maps that mHC is compared with: the unconstrained
+ * hyper-connections of the slavadubrov.com article, section "Kernmechanismen" (each map a
+ * static bias plus an input-dependent term through tanh, entries of either sign; its
+ * "Details van de parameterisatie" names tanh as what mHC replaces by the sigmoid).  The
+ * input-dependent term is the same normalised projection h that mhc_pre computes:
+ *   H_pre  = b_pre  + alpha_pre  * tanh(h[0:n])
+ *   H_res  = b_res  + alpha_res  * tanh(Mat(h[n:n+n^2]))      (no exp, no Sinkhorn)
+ *   H_post = b_post + alpha_post * tanh(h[n+n^2:m])
+ *   x_in   = sum_i H_pre[i] X_t[i, :]
+ * Same arguments, layouts, kernel paths and errors as mhc_pre_with_path, without t_max.
+ * mhc_post applies the result unchanged; mhc_amax_gain measures how its composite
+ * residual maps grow with depth, the comparison the pages draw.
+ */
+mhc_status mhc_pre_hc(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                      const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                      int64_t T, int n, int d, float eps, mhc_dtype dt, void* x_in, float* H,
+                      mhc_stream_t stream, mhc_pre_path path);
+
+/*
  * mhc_pre_path_for -- the path MHC_PRE_AUTO would take for this problem on the current
  * device (host-side query; launches nothing): MHC_PRE_CLUSTER_TC where it runs, else
  * MHC_PRE_GENERIC.

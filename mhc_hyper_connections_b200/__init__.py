@@ -8,6 +8,7 @@ CPU fallback -- if the library is missing the calls raise.
 
     mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,
             x_in, H)                -> writes x_in [T, d] and H [T, n*n+2n]
+    mhc_pre_hc(..., eps, x_in, H)   -> the same with the HC comparison maps (bias + alpha tanh)
     mhc_post(X, F_out, H, X_out)    -> writes X_out [T, n, d]
     mhc_pre_train(..., x_in, H, h)  -> mhc_pre plus the normalised projection h [T, m]
     mhc_backward(X, F_out, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
@@ -26,7 +27,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_post", "mhc_backward",
+__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_post", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "mhc_amax_gain", "mhc_pre_path_for", "mhc_device_status", "mhc_debug_pre_stop_after",
            "MhcError",
@@ -44,7 +45,7 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
            8: "MHC_ERR_WORKSPACE"}
 
 # Every function include/mhc.h declares.
-EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
+EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
                     "mhc_amax_gain", "mhc_status_string",
                     "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after")
@@ -81,6 +82,8 @@ def load_library():
         lib.mhc_pre.restype = ci
         lib.mhc_pre_with_path.argtypes = pre_args + [ci]
         lib.mhc_pre_with_path.restype = ci
+        lib.mhc_pre_hc.argtypes = pre_args[:12] + pre_args[13:] + [ci]
+        lib.mhc_pre_hc.restype = ci
         lib.mhc_pre_train.argtypes = pre_args[:-1] + [fp, vp]
         lib.mhc_pre_train.restype = ci
         lib.mhc_backward_workspace_bytes.argtypes = [i64, ci, ci]
@@ -177,6 +180,32 @@ def mhc_pre_with_path(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha
                                    float(alpha_res), T, n, d, float(eps), int(t_max), _dt(X),
                                    ptrs["x_in"], ptrs["H"], _stream(stream, dev), int(path))
     _check(st, "mhc_pre")
+
+
+def mhc_pre_hc(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, x_in, H,
+               stream=None, path: int = PRE_AUTO):
+    """Pre stage with the HC comparison maps: H = b + alpha tanh(h) for every coefficient
+    (no sigmoid, no Sinkhorn) and x_in = H_pre X; same shapes as mhc_pre."""
+    import torch
+    T, n, d = X.shape
+    dev = X.device
+    f32 = torch.float32
+    m = n * n + 2 * n
+    if tuple(phi.shape) != (n * d, m) or tuple(x_in.shape) != (T, d) or tuple(H.shape) != (T, m):
+        raise ValueError("mhc_pre_hc: shapes must be phi [n*d, m], x_in [T, d], H [T, m]")
+    if b_pre.numel() != n or b_post.numel() != n or b_res.numel() != n * n:
+        raise ValueError("mhc_pre_hc: b_pre/b_post need n entries, b_res n*n")
+    ptrs = dict(X=_ptr(X, "X", device=dev), phi=_ptr(phi, "phi", f32, dev),
+                b_pre=_ptr(b_pre, "b_pre", f32, dev), b_post=_ptr(b_post, "b_post", f32, dev),
+                b_res=_ptr(b_res, "b_res", f32, dev), x_in=_ptr(x_in, "x_in", X.dtype, dev),
+                H=_ptr(H, "H", f32, dev))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_pre_hc(ptrs["X"], ptrs["phi"], ptrs["b_pre"], ptrs["b_post"], ptrs["b_res"],
+                            float(alpha_pre), float(alpha_post), float(alpha_res), T, n, d,
+                            float(eps), _dt(X), ptrs["x_in"], ptrs["H"], _stream(stream, dev),
+                            int(path))
+    _check(st, "mhc_pre_hc")
 
 
 def mhc_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,

@@ -118,4 +118,20 @@ __device__ __forceinline__ void token_maps(const float* h, float inv_r, const fl
     (void)MM;
 }
 
+// The HC maps mHC is compared with (slavadubrov.com article, "Kernmechanismen": a static
+// bias plus an input-dependent term through tanh): every coefficient is
+// b + alpha * tanh(h / r), with no sigmoid, exp or Sinkhorn.  Same layout as token_maps.
+template <int N>
+__device__ __forceinline__ void token_maps_hc(const float* h, float inv_r, const float* b_pre,
+                                              const float* b_post, const float* b_res,
+                                              float a_pre, float a_post, float a_res, float* out) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = b_pre[i] + a_pre * tanhf(h[i] * inv_r);
+#pragma unroll
+    for (int k = 0; k < N * N; ++k) out[N + k] = b_res[k] + a_res * tanhf(h[N + k] * inv_r);
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+        out[N + N * N + i] = b_post[i] + a_post * tanhf(h[N + N * N + i] * inv_r);
+}
+
 }  // namespace mhc

@@ -23,6 +23,7 @@ struct PreArgs {
     void* x_in;
     float* H;
     float* h_out = nullptr;      // optional [T, m]: the normalised projection, for the backward
+    bool hc = false;             // HC maps (bias + alpha tanh) instead of mHC's
     cudaStream_t stream;
 };
 

@@ -125,7 +125,8 @@ mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
 static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, const float* b_post,
                            const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
                            int64_t T, int n, int d, float eps, int t_max, mhc_dtype dt, void* x_in,
-                           float* H, float* h_out, mhc_stream_t stream, mhc_pre_path path) {
+                           float* H, float* h_out, mhc_stream_t stream, mhc_pre_path path,
+                           bool hc = false) {
     mhc_status st = validate_pre(X, phi, b_pre, b_post, b_res, T, n, d, t_max, dt, x_in, H);
     if (st != MHC_OK) return st;
     if (path != MHC_PRE_AUTO && path != MHC_PRE_GENERIC && path != MHC_PRE_CLUSTER_TC)
@@ -135,6 +136,7 @@ static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, 
     PreArgs a = make_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T,
                          n, d, eps, t_max, dt, x_in, H, stream);
     a.h_out = h_out;
+    a.hc = hc;
     cudaError_t e;
     if (path == MHC_PRE_CLUSTER_TC) {
         if (!pre_tc_shape_ok(T, n, d, a.dt) || !pre_tc_device_ok(n, d))
@@ -156,6 +158,14 @@ mhc_status mhc_pre_with_path(const void* X, const float* phi, const float* b_pre
                              mhc_stream_t stream, mhc_pre_path path) {
     return pre_impl(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T, n, d, eps,
                     t_max, dt, x_in, H, nullptr, stream, path);
+}
+
+mhc_status mhc_pre_hc(const void* X, const float* phi, const float* b_pre, const float* b_post,
+                      const float* b_res, float alpha_pre, float alpha_post, float alpha_res,
+                      int64_t T, int n, int d, float eps, mhc_dtype dt, void* x_in, float* H,
+                      mhc_stream_t stream, mhc_pre_path path) {
+    return pre_impl(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T, n, d, eps,
+                    0, dt, x_in, H, nullptr, stream, path, true);
 }
 
 mhc_status mhc_pre_train(const void* X, const float* phi, const float* b_pre, const float* b_post,

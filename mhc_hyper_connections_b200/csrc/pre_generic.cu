@@ -5,7 +5,8 @@
 //      memory; accumulate the projection h = v . phi (fp32; each thread a TM-token by
 //      ceil(m/32)-column register tile) and the sum of squares of v.
 //   2. One thread per token turns h into [H_pre | H_res | H_post] ("DeepSeek-V4/mhc",
-//      equations rmsnorm, a/b/c-tilde, gate, sinkhorn) and writes H.
+//      equations rmsnorm, a/b/c-tilde, gate, sinkhorn; or the HC maps, bias + alpha tanh)
+//      and writes H.
 //   3. x_in = sum_i H_pre[i] X[t, i, :] (slavadubrov.com Eq. 3, read map on raw X).
 // Exact fp32 arithmetic with fp32 phi: this is the path for fp32 storage and for shapes
 // the tensor-core path does not take.
@@ -27,7 +28,7 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
                    const float* __restrict__ b_pre, const float* __restrict__ b_post,
                    const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                    int64_t Tn, int d, float eps, int t_max, T* __restrict__ x_in,
-                   float* __restrict__ H, float* __restrict__ h_out)
+                   float* __restrict__ H, float* __restrict__ h_out, int hc)
 {
     constexpr int M = N * N + 2 * N;
     constexpr int TJ = (M + JS - 1) / JS;              // columns per thread
@@ -117,7 +118,8 @@ pre_generic_kernel(const T* __restrict__ X, const float* __restrict__ phi,
         const float r = sqrtf(ss_s[tid] / (float)K + eps);
         float out[M];
         const float inv_r = 1.0f / r;
-        token_maps<N>(hs[tid], inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+        if (hc) token_maps_hc<N>(hs[tid], inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, out);
+        else token_maps<N>(hs[tid], inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
 #pragma unroll
         for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
         if (h_out != nullptr) {        // the normalised projection, as the logits use it
@@ -146,7 +148,7 @@ cudaError_t launch_n(const PreArgs& a) {
     if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
     pre_generic_kernel<N, T><<<(unsigned)blocks, THREADS, 0, a.stream>>>(
         static_cast<const T*>(a.X), a.phi, a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post,
-        a.a_res, a.T, a.d, a.eps, a.t_max, static_cast<T*>(a.x_in), a.H, a.h_out);
+        a.a_res, a.T, a.d, a.eps, a.t_max, static_cast<T*>(a.x_in), a.H, a.h_out, a.hc ? 1 : 0);
     return cudaGetLastError();
 }
 

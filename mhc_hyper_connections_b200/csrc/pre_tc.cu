@@ -23,7 +23,8 @@
 //   * The owner adds the 16 partials in a fixed order (deterministic, no atomics -- the
 //     property the paper's deterministic split-k provides, without split buffers in
 //     HBM), applies 1/r (RMSNorm after the projection), sends H_pre to all 16 CTAs, then
-//     runs Sinkhorn (H_res) and H_post for its tokens and writes H.
+//     runs Sinkhorn (H_res) and H_post for its tokens and writes H.  (The HC comparison
+//     maps take b + alpha tanh(h / r) for every coefficient instead.)
 //   * Eight warps form x_in for the CTA's share of the d channels once a tile's H_pre has
 //     arrived, re-reading that tile of X with plain loads: the tile was loaded moments
 //     before, so those reads hit L2 (the whole GPU keeps a few tiles per cluster, tens of
@@ -161,7 +162,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
               const float* __restrict__ b_post, const float* __restrict__ b_res, float a_pre,
               float a_post, float a_res, int T, int d, float eps, int t_max,
               __nv_bfloat16* __restrict__ x_in, float* __restrict__ H, float* __restrict__ h_out,
-              int ka_total, int ka_max, int nstage, int stop_tile, unsigned long long wait_ns)
+              int ka_total, int ka_max, int nstage, int stop_tile, unsigned long long wait_ns, int hc)
 {
     using C = Cfg<N>;
     constexpr int M = C::M, NB = C::NB, W = C::W;
@@ -438,11 +439,13 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 const float ssum = __shfl_sync(0xffffffffu, v[t], M);
                 const float inv_r = 1.0f / sqrtf(ssum * invK + eps);
                 const float hn = v[t] * inv_r;
-                const float z = alpha * hn + bias;
                 const int64_t tok = (int64_t)t0 + t * S + (int)rank;
                 if (h_out != nullptr && lane < M && tok < T) h_out[tok * M + lane] = hn;
-                hp[t] = lane < N ? sigmoid_f32(z) : 0.f;
-                if (lane < M) own[t * M + lane] = lane < N ? hp[t] : z;
+                // mHC: logit z, gates and (below) Sinkhorn; HC: the coefficient itself
+                const float z = hc ? bias + alpha * tanhf(hn) : alpha * hn + bias;
+                const float pre = hc ? z : sigmoid_f32(z);
+                hp[t] = lane < N ? pre : 0.f;
+                if (lane < M) own[t * M + lane] = lane < N ? pre : z;
             }
             // H_pre of the owner's tokens -> H_pre slot of every CTA of the cluster
             const int slh = k % NSLOT_H, uh = k / NSLOT_H;
@@ -460,7 +463,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             }
             __syncwarp();
             // Sinkhorn-Knopp (H_res) and H_post of the owner's tokens, one lane per token
-            if (lane < TPO) {
+            if (!hc && lane < TPO) {
                 float* L = own + lane * M;
                 float Mx[N][N];
 #pragma unroll
@@ -696,7 +699,7 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p) {
     return cudaLaunchKernelEx(&cfg, pre_tc_kernel<N>, maps, static_cast<const __nv_bfloat16*>(a.X), a.phi,
                               a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps,
                               a.t_max, static_cast<__nv_bfloat16*>(a.x_in), a.H, a.h_out, ka_total, p.ka_max,
-                              p.nstage, g_stop_tile.load(), g_wait_ns.load());
+                              p.nstage, g_stop_tile.load(), g_wait_ns.load(), a.hc ? 1 : 0);
 }
 
 }  // namespace tc
