@@ -25,14 +25,14 @@
 //     HBM), applies 1/r (RMSNorm after the projection), sends H_pre to all 16 CTAs, then
 //     runs Sinkhorn (H_res) and H_post for its tokens and writes H.  (The HC comparison
 //     maps take b + alpha tanh(h / r) for every coefficient instead.)
-//   * Eight warps form x_in for the CTA's share of the d channels once a tile's H_pre has
+//   * Six warps form x_in for the CTA's share of the d channels once a tile's H_pre has
 //     arrived, re-reading that tile of X with plain loads: the tile was loaded moments
 //     before, so those reads hit L2 (the whole GPU keeps a few tiles per cluster, tens of
 //     MB, in flight) and X still crosses HBM once.
 //
-// Warp roles (576 threads): 0 TMA producer and TMEM owner, 1 owner reduction / H, 2-3
-// and 16-17 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane
-// quarters 0-3), 8-15 x_in.  Every wait on an mbarrier is bounded in time; on expiry
+// Warp roles (512 threads): 0 TMA producer and TMEM owner, 1 owner reduction / H, 2-3
+// and 14-15 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane
+// quarters 0-3), 8-13 x_in.  Every wait on an mbarrier is bounded in time; on expiry
 // the kernel records the failing wait in a status word, drains its own copies in
 // flight, frees TMEM and returns.
 #include <cuda.h>
@@ -63,9 +63,9 @@ constexpr int NSLOT_P = 2;         // partial-projection receive slots
 constexpr int NSLOT_H = 2;         // H_pre receive slots
 constexpr int TPO = NT / S;        // tokens per owner per tile
 constexpr int MAXST = 4;           // max X stages
-constexpr int NXW = 8;             // x_in warps
+constexpr int NXW = 6;             // x_in warps
 constexpr int XU = 4;              // x_in tasks in flight per thread
-constexpr int NWARPS = 18;
+constexpr int NWARPS = 16;         // 4 warps per scheduler partition: up to 128 registers
 constexpr int THREADS = NWARPS * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int STAGE_BYTES = SA * NT * 128;      // 32 KB
@@ -156,7 +156,7 @@ struct Maps {
 
 // ---------------------------------------------------------------- the kernel
 template <int N>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(THREADS, 1)
 pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict__ X,
               const float* __restrict__ phi, const float* __restrict__ b_pre,
               const float* __restrict__ b_post, const float* __restrict__ b_res, float a_pre,
@@ -289,9 +289,9 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 drain(bar(B_FULL + j % nstage), (j / nstage) & 1, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3 || warp == 16 || warp == 17) {
+    } else if (warp == 2 || warp == 3 || warp >= 8 + NXW) {
         // MMA issuers: issuer i takes atom i of every stage, into accumulator i
-        const int i = warp < 4 ? warp - 2 : warp - 14;
+        const int i = warp < 4 ? warp - 2 : warp - (8 + NXW) + 2;
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_m64(NB);
             int g = 0, issued = 0;
