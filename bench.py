@@ -375,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
                     "gbs": by_pre * T / (pre_ms / 1e3) / 1e9,
                     "path": {1: "generic", 2: "cluster_tc"}.get(path, str(path)),
                     "source": "mhc_hyper_connections_b200/csrc/" +
-                              {2: "pre_cluster_tc.cu"}.get(path, "pre_generic.cu")},
+                              {2: "pre_tc.cu"}.get(path, "pre_generic.cu")},
             "post": {"ms": post_ms, "bytes_per_launch": by_post * T,
                      "gbs": by_post * T / (post_ms / 1e3) / 1e9,
                      "source": "mhc_hyper_connections_b200/csrc/post.cu"}}

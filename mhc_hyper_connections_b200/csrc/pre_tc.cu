@@ -22,17 +22,18 @@
 //     (local token t -> CTA t % 16) with one bulk shared-to-peer copy per owner.
 //   * The owner adds the 16 partials in a fixed order (deterministic, no atomics -- the
 //     property the paper's deterministic split-k provides, without split buffers in
-//     HBM), applies 1/r (RMSNorm after the projection), sends H_pre to all 16 CTAs, then
-//     runs Sinkhorn (H_res) and H_post for its tokens and writes H.  (The HC comparison
-//     maps take b + alpha tanh(h / r) for every coefficient instead.)
-//   * Six warps form x_in for the CTA's share of the d channels once a tile's H_pre has
+//     HBM), applies 1/r (RMSNorm after the projection) and sends H_pre to all 16 CTAs.
+//     A separate warp runs Sinkhorn (H_res) and H_post and writes H, one token per lane,
+//     32 tokens (8 tiles) per pass, off the critical path.  (The HC comparison maps take
+//     b + alpha tanh(h / r) for every coefficient instead.)
+//   * Five warps form x_in for the CTA's share of the d channels once a tile's H_pre has
 //     arrived, re-reading that tile of X with plain loads: the tile was loaded moments
 //     before, so those reads hit L2 (the whole GPU keeps a few tiles per cluster, tens of
 //     MB, in flight) and X still crosses HBM once.
 //
-// Warp roles (512 threads): 0 TMA producer and TMEM owner, 1 owner reduction / H, 2-3
-// and 14-15 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane
-// quarters 0-3), 8-13 x_in.  Every wait on an mbarrier is bounded in time; on expiry
+// Warp roles (512 threads): 0 TMA producer and TMEM owner, 1 owner reduction and H_pre,
+// 2-3 and 14-15 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane
+// quarters 0-3), 8-12 x_in, 13 Sinkhorn and the H store.  Every wait on an mbarrier is bounded in time; on expiry
 // the kernel records the failing wait in a status word, drains its own copies in
 // flight, frees TMEM and returns.
 #include <cuda.h>
@@ -63,8 +64,11 @@ constexpr int NSLOT_P = 2;         // partial-projection receive slots
 constexpr int NSLOT_H = 2;         // H_pre receive slots
 constexpr int TPO = NT / S;        // tokens per owner per tile
 constexpr int MAXST = 4;           // max X stages
-constexpr int NXW = 6;             // x_in warps
-constexpr int XU = 4;              // x_in tasks in flight per thread
+constexpr int NXW = 5;             // x_in warps
+constexpr int SK_WARP = 8 + NXW;   // Sinkhorn warp
+constexpr int BATCH = 32;          // tokens per Sinkhorn pass (one per lane)
+constexpr int RING = 2 * BATCH;    // logit ring: two passes
+constexpr int XU = 5;              // x_in tasks in flight per thread
 constexpr int NWARPS = 16;         // 4 warps per scheduler partition: up to 128 registers
 constexpr int THREADS = NWARPS * 32;
 constexpr int TMEM_COLS = 512;
@@ -72,6 +76,8 @@ constexpr int STAGE_BYTES = SA * NT * 128;      // 32 KB
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait, then give up
 
 static_assert(NMMA == SA, "one issuer per atom of a stage");
+static_assert(BATCH % TPO == 0, "a Sinkhorn pass holds whole tiles");
+static_assert(SK_WARP + 1 + NMMA - 2 == NWARPS, "warp roles fill the block");
 static_assert(NACC * NMMA * ACC_STRIDE <= TMEM_COLS, "accumulators fit TMEM");
 
 template <int N>
@@ -96,13 +102,15 @@ enum : int {
     B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = B_ACCF + NACC,
     B_PFULL = B_ACCE + NACC, B_PEMPTY = B_PFULL + NSLOT_P, B_HFULL = B_PEMPTY + NSLOT_P,
     B_HEMPTY = B_HFULL + NSLOT_H, B_DRAIN = B_HEMPTY + NSLOT_H, B_STG_FREE = B_DRAIN + NMMA,
-    B_STG_READY = B_STG_FREE + 1, B_XDONE = B_STG_READY + 1, B_COUNT = B_XDONE + NSLOT_H
+    B_STG_READY = B_STG_FREE + 1, B_XDONE = B_STG_READY + 1, B_LG_FULL = B_XDONE + NSLOT_H,
+    B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
 };
 
 // status codes: which wait expired
 enum : unsigned {
     E_EMPTY = 1u, E_FULL_MMA = 2u, E_ACCE = 4u, E_ACCF = 8u, E_PEMPTY = 16u, E_FULL_SS = 32u,
-    E_PFULL = 64u, E_HEMPTY = 128u, E_HFULL = 256u, E_DRAIN = 512u, E_STG = 1024u, E_XDONE = 2048u
+    E_PFULL = 64u, E_HEMPTY = 128u, E_HFULL = 256u, E_DRAIN = 512u, E_STG = 1024u, E_XDONE = 2048u,
+    E_LG_EMPTY = 4096u, E_LG_FULL = 8192u
 };
 
 using namespace ptx;
@@ -189,14 +197,14 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
     const uint32_t o_recv = off; off += (uint32_t)NSLOT_P * S * C::PART * 4u;
     const uint32_t o_stg = off;  off += (uint32_t)S * C::PART * 4u;
     const uint32_t o_hpre = off; off += (uint32_t)NSLOT_H * NT * 16u;
-    const uint32_t o_own = off;  off += (uint32_t)TPO * M * 4u;
+    const uint32_t o_ring = off; off += (uint32_t)RING * M * 4u;
     off = (off + 15u) & ~15u;
     const uint32_t o_bar = off;  off += B_COUNT * 8u;
     const uint32_t o_misc = off;
     float* recv = reinterpret_cast<float*>(sb + o_recv);
     float* stg = reinterpret_cast<float*>(sb + o_stg);
     float* hpre = reinterpret_cast<float*>(sb + o_hpre);
-    float* own = reinterpret_cast<float*>(sb + o_own);
+    float* ring = reinterpret_cast<float*>(sb + o_ring);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sb + o_misc);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sb + o_misc + 4);
     auto bar = [&](int i) -> uint32_t { return base + o_bar + 8u * (uint32_t)i; };
@@ -229,6 +237,10 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         mbar_init(bar(B_STG_FREE), 1);               // warp 4: the copies have read the staging block
         mbar_init(bar(B_STG_READY), 4);              // the 4 epilogue warps staged their rows
         for (int sl = 0; sl < NSLOT_H; ++sl) mbar_init(bar(B_XDONE + sl), NXW);   // x_in warps done
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_LG_FULL + b), 1);       // owner: a pass of logits is complete
+            mbar_init(bar(B_LG_EMPTY + b), 1);      // Sinkhorn warp: the pass is consumed
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -289,9 +301,9 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 drain(bar(B_FULL + j % nstage), (j / nstage) & 1, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3 || warp >= 8 + NXW) {
+    } else if (warp == 2 || warp == 3 || warp > SK_WARP) {
         // MMA issuers: issuer i takes atom i of every stage, into accumulator i
-        const int i = warp < 4 ? warp - 2 : warp - (8 + NXW) + 2;
+        const int i = warp < 4 ? warp - 2 : warp - (SK_WARP + 1) + 2;
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_m64(NB);
             int g = 0, issued = 0;
@@ -433,7 +445,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             __syncwarp();
             if (lane < S) mbar_arrive_remote(mapa(bar(B_PEMPTY + slot), (uint32_t)lane));
             const int t0 = (cid + k * ncl) * NT;
-            float hp[TPO];
+            float hp[TPO], zt[TPO];
 #pragma unroll
             for (int t = 0; t < TPO; ++t) {
                 const float ssum = __shfl_sync(0xffffffffu, v[t], M);
@@ -441,11 +453,11 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 const float hn = v[t] * inv_r;
                 const int64_t tok = (int64_t)t0 + t * S + (int)rank;
                 if (h_out != nullptr && lane < M && tok < T) h_out[tok * M + lane] = hn;
-                // mHC: logit z, gates and (below) Sinkhorn; HC: the coefficient itself
+                // mHC: logit z, gates and (Sinkhorn warp) Sinkhorn; HC: the coefficient itself
                 const float z = hc ? bias + alpha * tanhf(hn) : alpha * hn + bias;
                 const float pre = hc ? z : sigmoid_f32(z);
                 hp[t] = lane < N ? pre : 0.f;
-                if (lane < M) own[t * M + lane] = lane < N ? pre : z;
+                zt[t] = lane < N ? pre : z;
             }
             // H_pre of the owner's tokens -> H_pre slot of every CTA of the cluster
             const int slh = k % NSLOT_H, uh = k / NSLOT_H;
@@ -461,32 +473,52 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                                 mapa(bar(B_HFULL + slh), (uint32_t)lane));
                 }
             }
-            __syncwarp();
-            // Sinkhorn-Knopp (H_res) and H_post of the owner's tokens, one lane per token
-            if (!hc && lane < TPO) {
-                float* L = own + lane * M;
-                float Mx[N][N];
-#pragma unroll
-                for (int i = 0; i < N; ++i)
-#pragma unroll
-                    for (int j = 0; j < N; ++j) Mx[i][j] = expf(L[N + i * N + j]);
-                sinkhorn_rounds<N>(Mx, t_max);
-#pragma unroll
-                for (int i = 0; i < N; ++i)
-#pragma unroll
-                    for (int j = 0; j < N; ++j) L[N + i * N + j] = Mx[i][j];
-#pragma unroll
-                for (int i = 0; i < N; ++i) L[N + N * N + i] = 2.0f * sigmoid_f32(L[N + N * N + i]);
-            }
-            __syncwarp();
+            // [H_pre | res logits | post logits] of the owner's tokens -> the Sinkhorn ring;
+            // a pass is BATCH / TPO tiles
+            const int kb = k % (BATCH / TPO), pb = k / (BATCH / TPO), b = pb & 1;
+            if (kb == 0 && !wait(bar(B_LG_EMPTY + b), ((pb >> 1) & 1) ^ 1, E_LG_EMPTY)) break;
             if (lane < M) {
 #pragma unroll
-                for (int t = 0; t < TPO; ++t) {
-                    const int64_t tok = (int64_t)t0 + t * S + (int)rank;
-                    if (tok < T) H[tok * M + lane] = own[t * M + lane];
+                for (int t = 0; t < TPO; ++t) ring[(b * BATCH + kb * TPO + t) * M + lane] = zt[t];
+            }
+            __syncwarp();
+            if (lane == 0 && (kb == BATCH / TPO - 1 || k == my_tiles - 1)) mbar_arrive(bar(B_LG_FULL + b));
+        }
+    } else if (warp == SK_WARP) {
+        // Sinkhorn-Knopp (H_res), H_post and the H store: one token per lane, BATCH tokens
+        // (BATCH / TPO tiles of this owner) per pass
+        const int npass = (my_tiles + BATCH / TPO - 1) / (BATCH / TPO);
+        for (int pb = 0; pb < npass; ++pb) {
+            const int b = pb & 1;
+            if (!wait(bar(B_LG_FULL + b), (pb >> 1) & 1, E_LG_FULL)) break;
+            const int k = pb * (BATCH / TPO) + lane / TPO, t = lane % TPO;
+            if (k < my_tiles) {
+                const float* L = ring + (b * BATCH + lane) * M;
+                const int64_t tok = (int64_t)(cid + k * ncl) * NT + t * S + (int)rank;
+                float out[M];
+#pragma unroll
+                for (int j = 0; j < M; ++j) out[j] = L[j];
+                if (!hc) {
+                    float Mx[N][N];
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+#pragma unroll
+                        for (int j = 0; j < N; ++j) Mx[i][j] = expf(out[N + i * N + j]);
+                    sinkhorn_rounds<N>(Mx, t_max);
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+#pragma unroll
+                        for (int j = 0; j < N; ++j) out[N + i * N + j] = Mx[i][j];
+#pragma unroll
+                    for (int i = 0; i < N; ++i) out[N + N * N + i] = 2.0f * sigmoid_f32(out[N + N * N + i]);
+                }
+                if (tok < T) {
+#pragma unroll
+                    for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
                 }
             }
             __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_LG_EMPTY + b));
         }
     } else if (warp >= 8 && warp < 8 + NXW) {
         // x_in: task = (token t of the tile, 8-channel chunk c of this CTA's share)
@@ -566,7 +598,7 @@ template <int N>
 int smem_bytes(int ka_max, int nstage) {
     using C = Cfg<N>;
     int off = ka_max * C::PHI_ATOM + nstage * STAGE_BYTES + NSLOT_P * S * C::PART * 4 + S * C::PART * 4 +
-              NSLOT_H * NT * 16 + TPO * C::M * 4;
+              NSLOT_H * NT * 16 + RING * C::M * 4;
     off = (off + 15) & ~15;
     off += B_COUNT * 8 + 16;
     off += 1024;         // alignment slack of the dynamic shared-memory base
