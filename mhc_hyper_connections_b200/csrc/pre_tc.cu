@@ -138,16 +138,32 @@ struct Waiter {
     }
 };
 
-// 32 lanes x 8 consecutive 32-bit columns as floats, waiting for the load
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&f)[8]) {
-    uint32_t r[8];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
-                 "tcgen05.wait::ld.sync.aligned;"
+// TMEM -> registers without waiting (32 lanes x 8 or 16 consecutive columns); the registers
+// are valid only after tmem_wait_regs on them
+template <int W>
+__device__ __forceinline__ void tmem_ld_nowait(uint32_t taddr, uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_ld_nowait<8>(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7])
                  : "r"(taddr) : "memory");
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[i]);
+}
+template <>
+__device__ __forceinline__ void tmem_ld_nowait<16>(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr) : "memory");
+}
+// Wait for this thread's TMEM loads; the 8 registers are operands, so no use of them can be
+// scheduled before the wait
+__device__ __forceinline__ void tmem_wait_regs8(uint32_t* r) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]) :: "memory");
 }
 
 // streaming 16-byte read of X for the read map: the tile's last use, so L2 may drop it
@@ -374,17 +390,20 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             const int b = k % NACC, ub = k / NACC;
             if (!wait(bar(B_ACCF + b), ub & 1, E_ACCF)) break;
             tc_fence_after();
+            // one accumulator per round: all its columns in flight, then one wait
+            constexpr int LW = NB % 16 == 0 ? 16 : 8;
             float acc[NB];
 #pragma unroll
             for (int j = 0; j < NB; ++j) acc[j] = 0.f;
             for (int i = 0; i < nchain; ++i) {
+                uint32_t r[NB];
 #pragma unroll
-                for (int c8 = 0; c8 < NB / 8; ++c8) {
-                    float e[8];
-                    tmem_ld8(tq + (uint32_t)((b * NMMA + i) * ACC_STRIDE + c8 * 8), e);
+                for (int c = 0; c < NB / LW; ++c)
+                    tmem_ld_nowait<LW>(tq + (uint32_t)((b * NMMA + i) * ACC_STRIDE + c * LW), r + c * LW);
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) acc[c8 * 8 + x] += e[x];
-                }
+                for (int c8 = 0; c8 < NB / 8; ++c8) tmem_wait_regs8(r + c8 * 8);
+#pragma unroll
+                for (int j = 0; j < NB; ++j) acc[j] += __uint_as_float(r[j]);
             }
             tc_fence_before();
             __syncwarp();

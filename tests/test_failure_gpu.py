@@ -47,9 +47,9 @@ def test_expired_waits_are_reported_and_the_next_call_is_clean(restore_hook):
     code = mhc.mhc_device_status()
     assert code != 0
     assert mhc.mhc_device_status() == 0             # read-and-clear
-    # the tiles before the stop were finished: H is written for them, not for the rest
+    # the tiles before the stop were finished: x_in is written for them, not for the rest
     ref = run_oracle(w)
-    done = (H.abs().sum(dim=1) > 0).cpu().numpy()
+    done = (x_in.float().abs().sum(dim=1) > 0).cpu().numpy()
     assert done.any() and not done.all()
     mhc.mhc_debug_pre_stop_after(-1, 1_000_000)
     check_against_oracle(w, run_gpu(w, mhc.PRE_CLUSTER_TC, inputs=t), ref, "after expired waits")
