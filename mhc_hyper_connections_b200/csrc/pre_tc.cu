@@ -12,10 +12,10 @@
 //     128-byte swizzle.
 //   * Tokens stream through in tiles of NT = 64 (the MMA's M): one 3-D TMA box per stage
 //     copies SA = 4 atoms of 64 tokens (32 KB; large boxes are what lets one SM's TMA
-//     stream keep up with its share of HBM).  Four warps issue tcgen05.mma (M = 64,
-//     N = 2m, K = 16), atom j of a stage from issuer j, each into its own TMEM
-//     accumulator; the tensor core is then bound by its shared-memory operand reads
-//     (128 B per cycle), not by instruction issue.
+//     stream keep up with its share of HBM).  Two warps issue tcgen05.mma (M = 64,
+//     N = 2m, K = 16), atoms j, j + 2 of a stage from issuer j, each into its own TMEM
+//     accumulator (three buffers, so the MMAs of the next tiles do not wait for the
+//     epilogue).
 //   * The same four warps that read each stage for the tokens' sums of squares read the
 //     accumulators back (token t in TMEM lane 32 (t / 16) + t % 16), add hi + lo, and ship
 //     each token's partial projection and partial sum of squares to the token's owner CTA
@@ -26,14 +26,14 @@
 //     A separate warp runs Sinkhorn (H_res) and H_post and writes H, one token per lane,
 //     32 tokens (8 tiles) per pass, off the critical path.  (The HC comparison maps take
 //     b + alpha tanh(h / r) for every coefficient instead.)
-//   * Five warps form x_in for the CTA's share of the d channels once a tile's H_pre has
+//   * Seven warps form x_in for the CTA's share of the d channels once a tile's H_pre has
 //     arrived, re-reading that tile of X with plain loads: the tile was loaded moments
 //     before, so those reads hit L2 (the whole GPU keeps a few tiles per cluster, tens of
 //     MB, in flight) and X still crosses HBM once.
 //
 // Warp roles (512 threads): 0 TMA producer and TMEM owner, 1 owner reduction and H_pre,
-// 2-3 and 14-15 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane
-// quarters 0-3), 8-12 x_in, 13 Sinkhorn and the H store.  Every wait on an mbarrier is bounded in time; on expiry
+// 2-3 MMA issuers, 4-7 sums of squares and accumulator epilogue (TMEM lane quarters 0-3),
+// 8-14 x_in, 15 Sinkhorn and the H store.  Every wait on an mbarrier is bounded in time; on expiry
 // the kernel records the failing wait in a status word, drains its own copies in
 // flight, frees TMEM and returns.
 #include <cuda.h>
@@ -57,14 +57,14 @@ namespace tc {
 constexpr int S = 16;              // CTAs per cluster
 constexpr int NT = 64;             // tokens per tile = MMA M
 constexpr int SA = 4;              // 64-channel atoms per stage (TMA box depth)
-constexpr int NMMA = 4;            // MMA issuers: atom j of a stage goes to issuer j
-constexpr int NACC = 2;            // accumulator buffers (tile k -> buffer k % 2)
+constexpr int NMMA = 2;            // MMA issuers: atom j of a stage goes to issuer j % NMMA
+constexpr int NACC = 3;            // accumulator buffers (tile k -> buffer k % NACC)
 constexpr int ACC_STRIDE = 64;     // TMEM columns per accumulator
 constexpr int NSLOT_P = 2;         // partial-projection receive slots
 constexpr int NSLOT_H = 2;         // H_pre receive slots
 constexpr int TPO = NT / S;        // tokens per owner per tile
 constexpr int MAXST = 4;           // max X stages
-constexpr int NXW = 5;             // x_in warps
+constexpr int NXW = 7;             // x_in warps
 constexpr int SK_WARP = 8 + NXW;   // Sinkhorn warp
 constexpr int BATCH = 32;          // tokens per Sinkhorn pass (one per lane)
 constexpr int RING = 2 * BATCH;    // logit ring: two passes
@@ -75,9 +75,9 @@ constexpr int TMEM_COLS = 512;
 constexpr int STAGE_BYTES = SA * NT * 128;      // 32 KB
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait, then give up
 
-static_assert(NMMA == SA, "one issuer per atom of a stage");
+static_assert(SA % NMMA == 0, "every issuer gets the same atoms of a full stage");
 static_assert(BATCH % TPO == 0, "a Sinkhorn pass holds whole tiles");
-static_assert(SK_WARP + 1 + NMMA - 2 == NWARPS, "warp roles fill the block");
+static_assert(SK_WARP + 1 == NWARPS && NMMA == 2, "warp roles fill the block");
 static_assert(NACC * NMMA * ACC_STRIDE <= TMEM_COLS, "accumulators fit TMEM");
 
 template <int N>
@@ -317,9 +317,9 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 drain(bar(B_FULL + j % nstage), (j / nstage) & 1, E_DRAIN, false);
         }
         __syncwarp();
-    } else if (warp == 2 || warp == 3 || warp > SK_WARP) {
-        // MMA issuers: issuer i takes atom i of every stage, into accumulator i
-        const int i = warp < 4 ? warp - 2 : warp - (SK_WARP + 1) + 2;
+    } else if (warp == 2 || warp == 3) {
+        // MMA issuers: issuer i takes atoms i, i + NMMA, ... of every stage, into accumulator i
+        const int i = warp - 2;
         if (lane == 0) {
             constexpr uint32_t IDESC = idesc_m64(NB);
             int g = 0, issued = 0;
@@ -334,9 +334,9 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                     const int s = g % nstage, u = g / nstage;
                     if (!wait(bar(B_FULL + s), u & 1, E_FULL_MMA)) { stop = true; break; }
                     tc_fence_after();
-                    if (al + i < ka) {
-                        const uint64_t ad = sw128_desc(base + o_x + (uint32_t)s * STAGE_BYTES + (uint32_t)i * (NT * 128));
-                        const uint64_t bd = sw128_desc(base + o_phi + (uint32_t)(al + i) * C::PHI_ATOM);
+                    for (int j = i; j < SA && al + j < ka; j += NMMA) {
+                        const uint64_t ad = sw128_desc(base + o_x + (uint32_t)s * STAGE_BYTES + (uint32_t)j * (NT * 128));
+                        const uint64_t bd = sw128_desc(base + o_phi + (uint32_t)(al + j) * C::PHI_ATOM);
                         mma_bf16(d_tmem, ad, bd, IDESC, accumulate);
                         mma_bf16(d_tmem, ad + 2, bd + 2, IDESC, 1);
                         mma_bf16(d_tmem, ad + 4, bd + 4, IDESC, 1);
@@ -540,35 +540,47 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             if (lane == 0) mbar_arrive(bar(B_LG_EMPTY + b));
         }
     } else if (warp >= 8 && warp < 8 + NXW) {
-        // x_in: task = (token t of the tile, 8-channel chunk c of this CTA's share)
+        // x_in: this thread's tasks are xt, xt + NXT, ... of the tile's (token t, 8-channel
+        // chunk c of this CTA's share) pairs, walked with increments; a tile's first round
+        // of loads is issued before its H_pre arrives (the loads do not depend on it)
+        constexpr int NXT = NXW * 32;
         const int xt = threadIdx.x - 8 * 32;
         const uint64_t pol = policy_evict_first();
-        const int ntask = NT * nch;
+        const int st = NXT / nch, sc = NXT % nch;
+        const int t_first = xt / nch, c_first = xt % nch;
+        const int xrow = N * d;                      // elements of X per token
         for (int k = 0; k < my_tiles; ++k) {
             const int slh = k % NSLOT_H, uh = k / NSLOT_H;
-            if (!wait.template operator()<true>(bar(B_HFULL + slh), uh & 1, E_HFULL)) break;
             const int64_t t0 = (int64_t)(cid + k * ncl) * NT;
-            const float* hs = hpre + slh * NT * 4;
-            for (int task0 = xt; task0 < ntask; task0 += NXW * 32 * XU) {
-                uint4 xv[XU][N];
+            const int nt = T - t0 < NT ? (int)(T - t0) : NT;          // tokens of this tile
+            const __nv_bfloat16* xb = X + t0 * xrow + (int64_t)c_lo * 8;
+            __nv_bfloat16* ob = x_in + t0 * d + (int64_t)c_lo * 8;
+            int t = t_first, c = c_first;
+            uint4 xv[XU][N];
+            int tt[XU], cc[XU];
+            auto load_round = [&]() {
 #pragma unroll
                 for (int u = 0; u < XU; ++u) {
-                    const int task = task0 + u * NXW * 32;
-                    const int t = task / nch, c = c_lo + (task - t * nch);
-                    const int64_t tok = t0 + t;
-                    if (task < ntask && tok < T) {
-                        const __nv_bfloat16* src = X + (tok * N) * (int64_t)d + (int64_t)c * 8;
+                    tt[u] = t;
+                    cc[u] = c;
+                    if (t < nt) {
+                        const __nv_bfloat16* src = xb + (t * xrow + c * 8);
 #pragma unroll
-                        for (int i = 0; i < N; ++i) xv[u][i] = ld_last_use_v4(src + (int64_t)i * d, pol);
+                        for (int i = 0; i < N; ++i) xv[u][i] = ld_last_use_v4(src + i * d, pol);
                     }
+                    t += st;
+                    c += sc;
+                    if (c >= nch) { c -= nch; ++t; }
                 }
+            };
+            load_round();
+            if (!wait.template operator()<true>(bar(B_HFULL + slh), uh & 1, E_HFULL)) break;
+            const float* hs = hpre + slh * NT * 4;
+            while (true) {
 #pragma unroll
                 for (int u = 0; u < XU; ++u) {
-                    const int task = task0 + u * NXW * 32;
-                    const int t = task / nch, c = c_lo + (task - t * nch);
-                    const int64_t tok = t0 + t;
-                    if (task < ntask && tok < T) {
-                        const float4 h4 = *reinterpret_cast<const float4*>(hs + t * 4);
+                    if (tt[u] < nt) {
+                        const float4 h4 = *reinterpret_cast<const float4*>(hs + tt[u] * 4);
                         const float hv[4] = {h4.x, h4.y, h4.z, h4.w};
                         float acc[8];
 #pragma unroll
@@ -580,9 +592,11 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
 #pragma unroll
                             for (int e = 0; e < 8; ++e) acc[e] = fmaf(hv[i], f[e], acc[e]);
                         }
-                        st_v4(x_in + tok * d + (int64_t)c * 8, Vec16<__nv_bfloat16>::pack(acc));
+                        st_v4(ob + (tt[u] * d + cc[u] * 8), Vec16<__nv_bfloat16>::pack(acc));
                     }
                 }
+                if (t >= nt) break;
+                load_round();
             }
             // once every x_in warp is done with the slot, warp 8 arms its next phase and
             // releases it to the 16 owners
