@@ -64,6 +64,7 @@ constexpr int NSLOT_P = 2;         // partial-projection receive slots
 constexpr int NSLOT_H = 2;         // H_pre receive slots
 constexpr int TPO = NT / S;        // tokens per owner per tile
 constexpr int MAXST = 4;           // max X stages
+constexpr int PF = 4;              // stages of X prefetched into L2 ahead of their load
 constexpr int NXW = 7;             // x_in warps
 constexpr int SK_WARP = 8 + NXW;   // Sinkhorn warp
 constexpr int BATCH = 32;          // tokens per Sinkhorn pass (one per lane)
@@ -102,7 +103,7 @@ enum : int {
     B_FULL = 0, B_EMPTY = MAXST, B_ACCF = 2 * MAXST, B_ACCE = B_ACCF + NACC,
     B_PFULL = B_ACCE + NACC, B_PEMPTY = B_PFULL + NSLOT_P, B_HFULL = B_PEMPTY + NSLOT_P,
     B_HEMPTY = B_HFULL + NSLOT_H, B_DRAIN = B_HEMPTY + NSLOT_H, B_STG_FREE = B_DRAIN + NMMA,
-    B_STG_READY = B_STG_FREE + 1, B_XDONE = B_STG_READY + 1, B_LG_FULL = B_XDONE + NSLOT_H,
+    B_STG_READY = B_STG_FREE + 2, B_XDONE = B_STG_READY + 1, B_LG_FULL = B_XDONE + NSLOT_H,
     B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
 };
 
@@ -211,7 +212,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
     const uint32_t o_phi = off;  off += (uint32_t)ka_max * C::PHI_ATOM;
     const uint32_t o_x = off;    off += (uint32_t)nstage * STAGE_BYTES;
     const uint32_t o_recv = off; off += (uint32_t)NSLOT_P * S * C::PART * 4u;
-    const uint32_t o_stg = off;  off += (uint32_t)S * C::PART * 4u;
+    const uint32_t o_stg = off;  off += 2u * S * C::PART * 4u;     // two staging blocks
     const uint32_t o_hpre = off; off += (uint32_t)NSLOT_H * NT * 16u;
     const uint32_t o_ring = off; off += (uint32_t)RING * M * 4u;
     off = (off + 15u) & ~15u;
@@ -250,7 +251,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             mbar_init(bar(B_HEMPTY + sl), S);         // one remote arrive per CTA's x_in warps
         }
         for (int i = 0; i < NMMA; ++i) mbar_init(bar(B_DRAIN + i), 1);
-        mbar_init(bar(B_STG_FREE), 1);               // warp 4: the copies have read the staging block
+        for (int b = 0; b < 2; ++b) mbar_init(bar(B_STG_FREE + b), 1);   // warp 4: copies have read block b
         mbar_init(bar(B_STG_READY), 4);              // the 4 epilogue warps staged their rows
         for (int sl = 0; sl < NSLOT_H; ++sl) mbar_init(bar(B_XDONE + sl), NXW);   // x_in warps done
         for (int b = 0; b < 2; ++b) {
@@ -298,18 +299,38 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         // TMA producer: stage g of the CTA holds atoms [al, al + na) of one tile
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" :: "l"(&maps.box[SA - 1]) : "memory");
+            // stage g = (tile k = g / spt, atoms from al = (g % spt) * SA); the test hook stops
+            // every CTA at the same tile
+            const int spt = (ka + SA - 1) / SA;
+            const int ntile = stop_tile >= 0 && stop_tile < my_tiles ? stop_tile : my_tiles;
+            const int total = ntile * spt;
+            // the box of stage g: tile origin and first atom
+            auto stage_box = [&](int gg, int& t0, int& al, int& na) {
+                const int k = gg / spt;
+                al = (gg - k * spt) * SA;
+                na = ka - al < SA ? ka - al : SA;
+                t0 = (cid + k * ncl) * NT;
+            };
+            // L2 prefetch PF stages ahead: by the time a stage's load is issued its data is in
+            // L2, so a slot of the ring turns over in an L2 round trip, not an HBM one
+            for (int gg = 0; gg < PF && gg < total; ++gg) {
+                int t0, al, na;
+                stage_box(gg, t0, al, na);
+                tma_prefetch_3d(&maps.box[na - 1], 0, t0, a_lo + al);
+            }
             int g = 0;
-            bool stop = false;
-            for (int k = 0; k < my_tiles && !stop; ++k) {
-                if (k == stop_tile) break;           // test hook: every CTA stops at the same tile
-                const int t0 = (cid + k * ncl) * NT;
-                for (int al = 0; al < ka; al += SA, ++g) {
-                    const int na = ka - al < SA ? ka - al : SA;
-                    const int s = g % nstage, u = g / nstage;
-                    if (!wait(bar(B_EMPTY + s), (u & 1) ^ 1, E_EMPTY)) { stop = true; break; }
-                    mbar_arrive_tx(bar(B_FULL + s), (uint32_t)(na * NT * 128));
-                    tma_load_3d(base + o_x + (uint32_t)s * STAGE_BYTES, &maps.box[na - 1], bar(B_FULL + s),
-                                0, t0, a_lo + al);
+            for (; g < total; ++g) {
+                int t0, al, na;
+                stage_box(g, t0, al, na);
+                const int s = g % nstage, u = g / nstage;
+                if (!wait(bar(B_EMPTY + s), (u & 1) ^ 1, E_EMPTY)) break;
+                mbar_arrive_tx(bar(B_FULL + s), (uint32_t)(na * NT * 128));
+                tma_load_3d(base + o_x + (uint32_t)s * STAGE_BYTES, &maps.box[na - 1], bar(B_FULL + s),
+                            0, t0, a_lo + al);
+                if (g + PF < total) {
+                    int pt0, pal, pna;
+                    stage_box(g + PF, pt0, pal, pna);
+                    tma_prefetch_3d(&maps.box[pna - 1], 0, pt0, a_lo + pal);
                 }
             }
             // drain: every issued copy has landed before the CTA can leave
@@ -408,11 +429,13 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_ACCE + b));
-            // stage [h partial (hi + lo) | sum of squares] for the token's owner (lane % 16),
-            // once tile k-1's copies have read the staging block
-            if (!wait(bar(B_STG_FREE), (k & 1) ^ 1, E_STG)) break;
+            // stage [h partial (hi + lo) | sum of squares] for the token's owner (lane % 16) in
+            // block k % 2, once tile k-2's copies have read it
+            const int sb2 = k & 1;
+            float* stgk = stg + sb2 * S * C::PART;
+            if (!wait(bar(B_STG_FREE + sb2), ((k >> 1) & 1) ^ 1, E_STG)) break;
             if (lane < 16) {
-                float* dst = stg + (lane * TPO + q) * W;
+                float* dst = stgk + (lane * TPO + q) * W;
 #pragma unroll
                 for (int j = 0; j < M; ++j) dst[j] = acc[j] + acc[M + j];
                 dst[M] = ss;
@@ -427,13 +450,13 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                     const int slot = k % NSLOT_P, us = k / NSLOT_P;
                     if (wait(bar(B_PEMPTY + slot), (us & 1) ^ 1, E_PEMPTY)) {
                         const uint32_t dst = base + o_recv + (uint32_t)((slot * S + (int)rank) * C::PART) * 4u;
-                        bulk_to_peer(mapa(dst, (uint32_t)lane), smem_u32(stg + lane * C::PART),
+                        bulk_to_peer(mapa(dst, (uint32_t)lane), smem_u32(stgk + lane * C::PART),
                                      (uint32_t)(C::PART * 4), mapa(bar(B_PFULL + slot), (uint32_t)lane));
                     }
-                    bulk_wait_read_all();
+                    bulk_wait_read_allbut1();     // tile k-1's copies have read their block
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_STG_FREE));
+                if (lane == 0 && k > 0) mbar_arrive(bar(B_STG_FREE + (sb2 ^ 1)));
             }
         }
         if (q == 0 && lane < S) bulk_wait_all();
@@ -630,7 +653,7 @@ struct Plan {
 template <int N>
 int smem_bytes(int ka_max, int nstage) {
     using C = Cfg<N>;
-    int off = ka_max * C::PHI_ATOM + nstage * STAGE_BYTES + NSLOT_P * S * C::PART * 4 + S * C::PART * 4 +
+    int off = ka_max * C::PHI_ATOM + nstage * STAGE_BYTES + NSLOT_P * S * C::PART * 4 + 2 * S * C::PART * 4 +
               NSLOT_H * NT * 16 + RING * C::M * 4;
     off = (off + 15) & ~15;
     off += B_COUNT * 8 + 16;

@@ -158,6 +158,11 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
                  " [%0], [%1, {%2, %3, %4}], [%5], %6;"
                  :: "r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy) : "memory");
 }
+// 3-D tiled prefetch of a box into L2 (no shared memory, no completion to wait for)
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 :: "l"(map), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
 // 4-D tiled TMA load
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
