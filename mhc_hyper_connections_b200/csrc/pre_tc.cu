@@ -384,28 +384,36 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         int g = 0;
         for (int k = 0; k < my_tiles; ++k) {
-            float ss = 0.f;
+            float sv[8];                          // eight independent FMA chains
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sv[e] = 0.f;
             bool ok = true;
             for (int al = 0; al < ka; al += SA, ++g) {
                 const int na = ka - al < SA ? ka - al : SA;
                 const int s = g % nstage, u = g / nstage;
                 if (!wait(bar(B_FULL + s), u & 1, E_FULL_SS)) { ok = false; break; }
                 const uint8_t* xs = sb + o_x + (uint32_t)s * STAGE_BYTES + (uint32_t)row * 128;
-                for (int a = 0; a < na; ++a) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const int j = half * 4 + kk;
-                        const uint4 w = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + ((j ^ (row & 7)) << 4));
-                        float f[8];
-                        Vec16<__nv_bfloat16>::unpack(w, f);
+                for (int a = 0; a < SA; ++a) {
+                    if (a < na) {
+                        uint4 w[4];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                        for (int kk = 0; kk < 4; ++kk)
+                            w[kk] = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + (((half * 4 + kk) ^ (row & 7)) << 4));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            float f[8];
+                            Vec16<__nv_bfloat16>::unpack(w[kk], f);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) sv[e] = fmaf(f[e], f[e], sv[e]);
+                        }
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
             }
             if (!ok) break;
+            float ss = ((sv[0] + sv[1]) + (sv[2] + sv[3])) + ((sv[4] + sv[5]) + (sv[6] + sv[7]));
             ss += __shfl_xor_sync(0xffffffffu, ss, 16);
             // accumulators of tile k: sum the issuers' partial projections
             const int b = k % NACC, ub = k / NACC;
