@@ -64,7 +64,7 @@ constexpr int NSLOT_P = 2;         // partial-projection receive slots
 constexpr int NSLOT_H = 2;         // H_pre receive slots
 constexpr int TPO = NT / S;        // tokens per owner per tile
 constexpr int MAXST = 4;           // max X stages
-constexpr int PF = 4;              // stages of X prefetched into L2 ahead of their load
+constexpr int PF = 0;              // stages of X prefetched into L2 ahead of their load (measured: none is best)
 constexpr int NXW = 7;             // x_in warps
 constexpr int SK_WARP = 8 + NXW;   // Sinkhorn warp
 constexpr int BATCH = 32;          // tokens per Sinkhorn pass (one per lane)
@@ -78,6 +78,7 @@ constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s per wait, then gi
 
 static_assert(SA % NMMA == 0, "every issuer gets the same atoms of a full stage");
 static_assert(BATCH % TPO == 0, "a Sinkhorn pass holds whole tiles");
+static_assert(BATCH == 32, "the Sinkhorn warp takes one token of a pass per lane");
 static_assert(SK_WARP + 1 == NWARPS && NMMA == 2, "warp roles fill the block");
 static_assert(NACC * NMMA * ACC_STRIDE <= TMEM_COLS, "accumulators fit TMEM");
 
