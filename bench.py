@@ -321,8 +321,8 @@ def run_ours(args, rank, world, local_rank):
                          Y=torch.empty_like(Xi)))
     X, F, x_in, H, Y = (bufs[0][k] for k in ("X", "F", "x_in", "H", "Y"))
     s = w.scalars()
-    req = {"auto": mhc.PRE_AUTO, "generic": mhc.PRE_GENERIC,
-           "cluster_tc": mhc.PRE_CLUSTER_TC}[args.pre_path]
+    req = {"auto": mhc.PRE_AUTO, "generic": mhc.PRE_GENERIC, "cluster_tc": mhc.PRE_CLUSTER_TC,
+           "two_pass_tc": mhc.PRE_TWO_PASS_TC}[args.pre_path]
     path = mhc.mhc_pre_path_for(T, n, d, tdt) if req == mhc.PRE_AUTO else req
 
     def pre(k=0):
@@ -373,9 +373,9 @@ def run_ours(args, rank, world, local_rank):
     by_pre, by_post = bytes_per_token(n, d, es)
     kern = {"pre": {"ms": pre_ms, "bytes_per_launch": by_pre * T,
                     "gbs": by_pre * T / (pre_ms / 1e3) / 1e9,
-                    "path": {1: "generic", 2: "cluster_tc"}.get(path, str(path)),
+                    "path": {1: "generic", 2: "cluster_tc", 3: "two_pass_tc"}.get(path, str(path)),
                     "source": "mhc_hyper_connections_b200/csrc/" +
-                              {2: "pre_tc.cu"}.get(path, "pre_generic.cu")},
+                              {2: "pre_tc.cu", 3: "pre_wide.cu"}.get(path, "pre_generic.cu")},
             "post": {"ms": post_ms, "bytes_per_launch": by_post * T,
                      "gbs": by_post * T / (post_ms / 1e3) / 1e9,
                      "source": "mhc_hyper_connections_b200/csrc/post.cu"}}
@@ -646,7 +646,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--pre-path", default="auto",
-                    choices=["auto", "generic", "cluster_tc"],
+                    choices=["auto", "generic", "cluster_tc", "two_pass_tc"],
                     help="kernel path of the pre stage (default: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)

@@ -81,9 +81,14 @@ typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
 typedef enum {
     MHC_PRE_AUTO = 0,          /* the fastest path that supports the problem          */
     MHC_PRE_GENERIC = 1,       /* CUDA-core kernel: any n <= 8, any d, f32 or bf16    */
-    MHC_PRE_CLUSTER_TC = 2     /* thread-block-cluster tensor-core kernel (bf16,      */
-                               /* n <= 4, d % 64 == 0, n*d >= 1024, phi slice fits    */
-                               /* shared memory, e.g. d <= 6144 at n = 4; sm_100)     */
+    MHC_PRE_CLUSTER_TC = 2,    /* thread-block-cluster tensor-core kernel, X read     */
+                               /* once (bf16, n <= 4, d % 64 == 0, n*d >= 1024, phi   */
+                               /* slice fits shared memory: d <= 5632 at n = 4)       */
+    MHC_PRE_TWO_PASS_TC = 3    /* tensor-core projection, then a streaming read map   */
+                               /* (X read twice; bf16, n <= 8, d % 64 == 0,           */
+                               /* n*d >= 512, and x_in large enough to hold phi       */
+                               /* packed for the MMA plus the partial projections --  */
+                               /* it is used as scratch before x_in is written)       */
 } mhc_pre_path;
 
 /*
@@ -140,9 +145,17 @@ mhc_status mhc_pre_hc(const void* X, const float* phi, const float* b_pre, const
 /*
  * mhc_pre_path_for -- the path MHC_PRE_AUTO would take for this problem on the current
  * device (host-side query; launches nothing): MHC_PRE_CLUSTER_TC where it runs, else
- * MHC_PRE_GENERIC.
+ * MHC_PRE_TWO_PASS_TC where it runs, else MHC_PRE_GENERIC.  The tensor-core paths also
+ * need X, x_in and phi 16-byte aligned; MHC_PRE_AUTO takes MHC_PRE_GENERIC when they are not.
  */
 mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt);
+
+/*
+ * mhc_pre_path_ok -- 1 if `path` can run a pre stage of this shape and storage type on the
+ * current device (given 16-byte-aligned X, x_in and phi for the tensor-core paths), else 0.
+ * MHC_PRE_AUTO and MHC_PRE_GENERIC run every valid shape.  Host-side, launches nothing.
+ */
+int mhc_pre_path_ok(int64_t T, int n, int d, mhc_dtype dt, mhc_pre_path path);
 
 /*
  * mhc_post -- the post/res merge for T tokens (slavadubrov.com Eq. 3, first and second
@@ -259,8 +272,8 @@ mhc_status mhc_amax_gain(const float* H_layers, int L, int64_t T, int n, float* 
                          mhc_stream_t stream);
 
 /*
- * mhc_device_status -- read and clear the device-side status word of the tensor-core
- * kernel.  Its waits between warps and between the CTAs of a cluster are bounded in
+ * mhc_device_status -- read and clear the device-side status words of the tensor-core
+ * kernels.  Their waits between warps and between the CTAs of a cluster are bounded in
  * time (1 s each); a wait that expires makes the kernel stop early, leaving its outputs
  * incomplete, and sets a bit here naming the wait.  *code = 0 means every wait of every
  * launch since the last read completed.  Blocks until prior work on the legacy default

@@ -29,9 +29,10 @@ import threading
 
 __all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_post", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
-           "mhc_amax_gain", "mhc_pre_path_for", "mhc_device_status", "mhc_debug_pre_stop_after",
+           "mhc_amax_gain", "mhc_pre_path_for", "mhc_pre_path_ok", "mhc_device_status",
+           "mhc_debug_pre_stop_after",
            "MhcError",
-           "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "library_path",
+           "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "PRE_TWO_PASS_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -39,13 +40,14 @@ _LIB_PATH = os.path.join(_HERE, "libmhc_b200.so")
 
 MHC_F32, MHC_BF16 = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20      # the fixed scratch array of mhc_backward_noalloc
-PRE_AUTO, PRE_GENERIC, PRE_CLUSTER_TC = 0, 1, 2
+PRE_AUTO, PRE_GENERIC, PRE_CLUSTER_TC, PRE_TWO_PASS_TC = 0, 1, 2, 3
 _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN",
            4: "MHC_ERR_DTYPE", 5: "MHC_ERR_UNSUPPORTED", 6: "MHC_ERR_CUDA", 7: "MHC_ERR_ALIAS",
            8: "MHC_ERR_WORKSPACE"}
 
 # Every function include/mhc.h declares.
-EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_pre_path_for", "mhc_post",
+EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_pre_path_for",
+                    "mhc_pre_path_ok", "mhc_post",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
                     "mhc_amax_gain", "mhc_status_string",
                     "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after")
@@ -97,6 +99,8 @@ def load_library():
         lib.mhc_amax_gain.restype = ci
         lib.mhc_pre_path_for.argtypes = [i64, ci, ci, ci]
         lib.mhc_pre_path_for.restype = ci
+        lib.mhc_pre_path_ok.argtypes = [i64, ci, ci, ci, ci]
+        lib.mhc_pre_path_ok.restype = ci
         lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
         lib.mhc_post.restype = ci
         lib.mhc_status_string.argtypes = [ci]
@@ -388,8 +392,16 @@ def mhc_debug_pre_stop_after(tiles: int, wait_limit_us: int = 1_000_000) -> None
            "mhc_debug_pre_stop_after")
 
 
+def mhc_pre_path_ok(T: int, n: int, d: int, dtype, path: int) -> bool:
+    """Whether kernel path `path` can run this shape on the current device."""
+    import torch
+    dt = dtype if isinstance(dtype, int) else (MHC_BF16 if dtype == torch.bfloat16 else MHC_F32)
+    return bool(load_library().mhc_pre_path_ok(int(T), int(n), int(d), dt, int(path)))
+
+
 def mhc_pre_path_for(T: int, n: int, d: int, dtype) -> int:
-    """Kernel path mhc_pre would take on the current device (PRE_GENERIC or PRE_CLUSTER_TC)."""
+    """Kernel path mhc_pre would take on the current device (PRE_GENERIC, PRE_CLUSTER_TC or
+    PRE_TWO_PASS_TC)."""
     import torch
     dt = dtype if isinstance(dtype, int) else (MHC_BF16 if dtype == torch.bfloat16 else MHC_F32)
     return int(load_library().mhc_pre_path_for(int(T), int(n), int(d), dt))

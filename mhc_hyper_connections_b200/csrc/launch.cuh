@@ -61,6 +61,14 @@ cudaError_t pre_tc_status(unsigned* out, bool clear);
 // per cluster (< 0: never) and give up a wait after `wait_ns`.
 void pre_tc_set_stop(int stop_tile, unsigned long long wait_ns);
 
+// Two-pass tensor-core path (8-CTA clusters, phi packed into the x_in buffer): shapes whose phi
+// slice does not fit one 16-CTA cluster (n = 5..8, or n <= 4 with a large d).  The shape test
+// includes the x_in buffer being large enough to hold the packed phi and the partials.
+bool pre_wide_shape_ok(int64_t T, int n, int d, DType dt);
+bool pre_wide_device_ok(int n);
+cudaError_t launch_pre_wide(const PreArgs& a);
+cudaError_t pre_wide_status(unsigned* out, bool clear);
+
 cudaError_t launch_post(const PostArgs& a);
 
 // Reverse mode of pre + post (backward.cu).

@@ -119,7 +119,20 @@ mhc_pre_path mhc_pre_path_for(int64_t T, int n, int d, mhc_dtype dt) {
     if (check_shape(T, n, d, dt) != MHC_OK) return MHC_PRE_GENERIC;
     const DType t = dt == MHC_BF16 ? BF16 : F32;
     if (pre_tc_shape_ok(T, n, d, t) && pre_tc_device_ok(n, d)) return MHC_PRE_CLUSTER_TC;
+    if (pre_wide_shape_ok(T, n, d, t) && pre_wide_device_ok(n)) return MHC_PRE_TWO_PASS_TC;
     return MHC_PRE_GENERIC;
+}
+
+int mhc_pre_path_ok(int64_t T, int n, int d, mhc_dtype dt, mhc_pre_path path) {
+    if (check_shape(T, n, d, dt) != MHC_OK) return 0;
+    const DType t = dt == MHC_BF16 ? BF16 : F32;
+    switch (path) {
+        case MHC_PRE_AUTO:
+        case MHC_PRE_GENERIC: return 1;
+        case MHC_PRE_CLUSTER_TC: return pre_tc_shape_ok(T, n, d, t) && pre_tc_device_ok(n, d);
+        case MHC_PRE_TWO_PASS_TC: return pre_wide_shape_ok(T, n, d, t) && pre_wide_device_ok(n);
+    }
+    return 0;
 }
 
 static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, const float* b_post,
@@ -129,21 +142,30 @@ static mhc_status pre_impl(const void* X, const float* phi, const float* b_pre, 
                            bool hc = false) {
     mhc_status st = validate_pre(X, phi, b_pre, b_post, b_res, T, n, d, t_max, dt, x_in, H);
     if (st != MHC_OK) return st;
-    if (path != MHC_PRE_AUTO && path != MHC_PRE_GENERIC && path != MHC_PRE_CLUSTER_TC)
+    if (path != MHC_PRE_AUTO && path != MHC_PRE_GENERIC && path != MHC_PRE_CLUSTER_TC &&
+        path != MHC_PRE_TWO_PASS_TC)
         return MHC_ERR_UNSUPPORTED;
     if (T == 0) return MHC_OK;
-    if (path == MHC_PRE_AUTO) path = mhc_pre_path_for(T, n, d, dt);
+    const bool tc_aligned = aligned(X, 16) && aligned(x_in, 16) && aligned(phi, 16);
+    if (path == MHC_PRE_AUTO) {
+        path = mhc_pre_path_for(T, n, d, dt);
+        if (path != MHC_PRE_GENERIC && !tc_aligned) path = MHC_PRE_GENERIC;
+    }
     PreArgs a = make_pre(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, T,
                          n, d, eps, t_max, dt, x_in, H, stream);
     a.h_out = h_out;
     a.hc = hc;
     cudaError_t e;
     if (path == MHC_PRE_CLUSTER_TC) {
-        if (!pre_tc_shape_ok(T, n, d, a.dt) || !pre_tc_device_ok(n, d))
+        if (!pre_tc_shape_ok(T, n, d, a.dt) || !pre_tc_device_ok(n, d) || !tc_aligned)
             return MHC_ERR_UNSUPPORTED;
-        if (!aligned(X, 16) || !aligned(x_in, 16) || !aligned(phi, 16)) return MHC_ERR_UNSUPPORTED;
         e = launch_pre_tc(a);
         if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (tensor-core kernel)");
+    } else if (path == MHC_PRE_TWO_PASS_TC) {
+        if (!pre_wide_shape_ok(T, n, d, a.dt) || !pre_wide_device_ok(n) || !tc_aligned)
+            return MHC_ERR_UNSUPPORTED;
+        e = launch_pre_wide(a);
+        if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (two-pass tensor-core kernels)");
     } else {
         e = launch_pre_generic(a);
         if (e != cudaSuccess) return cuda_fail(e, "mhc_pre (generic kernel)");
@@ -326,10 +348,11 @@ mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us) {
 
 mhc_status mhc_device_status(uint32_t* code) {
     if (!code) return MHC_ERR_NULL;
-    unsigned v = 0;
+    unsigned v = 0, w = 0;
     cudaError_t e = pre_tc_status(&v, true);
+    if (e == cudaSuccess) e = pre_wide_status(&w, true);
     if (e != cudaSuccess) return cuda_fail(e, "mhc_device_status");
-    *code = v;
+    *code = v | (w << 16);
     return MHC_OK;
 }
 

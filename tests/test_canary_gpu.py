@@ -4,8 +4,8 @@ Every output of mhc_pre, mhc_pre_train, mhc_post, mhc_backward (its workspace in
 and mhc_amax_gain is a view with GUARD bytes of a fixed pattern before and after it.
 After the call both guards must be intact, and the outputs must equal, bit for bit, those
 of the same call on plain tensors (every kernel here is deterministic).  The shapes are
-those of the parity tests: ragged token tails, odd d, both pre paths and both post
-kernels."""
+those of the parity tests: ragged token tails, odd d, all three pre paths (the two-pass
+tensor-core path uses x_in as scratch before writing it) and both post kernels."""
 import numpy as np
 import pytest
 
@@ -45,7 +45,8 @@ def _same_and_intact(plain, guarded, bufs):
 
 @pytest.mark.parametrize("T,n,d,dt", [(1, 4, 64, "bf16"), (17, 4, 1024, "bf16"), (19, 3, 40, "f32"),
                                       (9, 8, 64, "f32"), (3, 4, 37, "bf16"), (100, 4, 2048, "bf16"),
-                                      (130, 4, 4096, "bf16"), (40, 1, 1024, "bf16")])
+                                      (130, 4, 4096, "bf16"), (40, 1, 1024, "bf16"), (77, 4, 2560, "bf16"),
+                                      (2000, 8, 4096, "bf16"), (400, 4, 8192, "bf16")])
 def test_forward_writes_stay_inside_their_outputs(T, n, d, dt):
     w = wl.make_inputs(T=T, n=n, d=d, dtype=dt, seed=T + n + d, outlier_frac=0.01)
     t = torch_inputs(w, device=DEV)

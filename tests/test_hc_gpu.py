@@ -19,10 +19,9 @@ pytestmark = pytest.mark.gpu
 
 
 def _paths(w):
-    paths = [mhc.PRE_GENERIC]
-    if mhc.mhc_pre_path_for(w.T, w.n, w.d, 1 if w.dtype == "bf16" else 0) == mhc.PRE_CLUSTER_TC:
-        paths.append(mhc.PRE_CLUSTER_TC)
-    return paths
+    dt = 1 if w.dtype == "bf16" else 0
+    return [p for p in (mhc.PRE_GENERIC, mhc.PRE_CLUSTER_TC, mhc.PRE_TWO_PASS_TC)
+            if mhc.mhc_pre_path_ok(w.T, w.n, w.d, dt, p)]
 
 
 def run_gpu_hc(w, path, inputs=None):
@@ -62,7 +61,8 @@ def _hc_inputs(T, n, d, dtype, seed, alpha):
 @pytest.mark.parametrize("T,n,d,dt,alpha", [
     (64, 4, 64, "f32", 0.3), (4096, 4, 1024, "bf16", 0.01), (130, 4, 4096, "bf16", 0.5),
     (77, 4, 2560, "bf16", 1.0), (33, 1, 1024, "bf16", 0.7), (50, 3, 1280, "bf16", 0.4),
-    (19, 8, 64, "bf16", 0.5), (9, 2, 24, "f32", 0.9),
+    (19, 8, 64, "bf16", 0.5), (9, 2, 24, "f32", 0.9), (2000, 8, 4096, "bf16", 0.5),
+    (400, 4, 8192, "bf16", 0.8),
 ])
 def test_hc_maps_match_the_oracle(T, n, d, dt, alpha):
     w = _hc_inputs(T, n, d, dt, seed=T + 10 * n + d, alpha=alpha)

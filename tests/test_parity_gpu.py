@@ -19,10 +19,9 @@ pytestmark = pytest.mark.gpu
 
 def _paths(w):
     """Every pre path that can run this workload on this device."""
-    paths = [mhc.PRE_GENERIC]
-    if mhc.mhc_pre_path_for(w.T, w.n, w.d, 1 if w.dtype == "bf16" else 0) == mhc.PRE_CLUSTER_TC:
-        paths.append(mhc.PRE_CLUSTER_TC)
-    return paths
+    dt = 1 if w.dtype == "bf16" else 0
+    return [p for p in (mhc.PRE_GENERIC, mhc.PRE_CLUSTER_TC, mhc.PRE_TWO_PASS_TC)
+            if mhc.mhc_pre_path_ok(w.T, w.n, w.d, dt, p)]
 
 
 def test_library_is_the_one_in_tree():
@@ -106,6 +105,10 @@ SHAPES = [  # (T, n, d, dtype): ragged token tails, odd d, every n
     # tensor-core path at channel counts off the powers of two, several tiles per cluster
     (77, 4, 2560, "bf16"), (65, 4, 5120, "bf16"), (1363, 4, 512, "bf16"), (200, 3, 1280, "bf16"),
     (129, 2, 768, "bf16"), (1000, 1, 1024, "bf16"), (64 * 7 * 3 + 17, 4, 1024, "bf16"),
+    # two-pass tensor-core path: n = 5..8, and d past the cluster kernel's shared memory
+    (2000, 8, 4096, "bf16"), (2100, 7, 2048, "bf16"), (1500, 6, 1536, "bf16"),
+    (2100, 5, 1024, "bf16"), (400, 4, 8192, "bf16"), (350, 4, 7168, "bf16"), (300, 4, 6144, "bf16"),
+    (1300, 4, 2048, "bf16"), (700, 3, 1024, "bf16"),
 ]
 
 
@@ -208,8 +211,9 @@ def test_paths_agree_with_each_other():
 
 def test_auto_path_on_b200_shapes_is_tensor_core():
     """On a B200 the bf16 shapes with n <= 4, d a multiple of 64, n*d >= 1024 and a phi slice
-    that fits shared memory run the cluster tensor-core kernel; everything else runs the
-    generic kernel."""
+    that fits shared memory run the cluster tensor-core kernel; other bf16 shapes up to n = 8
+    whose x_in buffer can hold the packed phi run the two-pass tensor-core kernels; the rest
+    runs the generic kernel."""
     major, minor = torch.cuda.get_device_capability()
     if (major, minor) != (10, 0):
         pytest.skip("not an sm_100 device")
@@ -218,7 +222,10 @@ def test_auto_path_on_b200_shapes_is_tensor_core():
             assert mhc.mhc_pre_path_for(16384, n, d, 1) == mhc.PRE_CLUSTER_TC, (n, d)
     assert mhc.mhc_pre_path_for(16384, 4, 512, 1) == mhc.PRE_CLUSTER_TC       # n*d = 2048
     assert mhc.mhc_pre_path_for(16384, 4, 4096, 0) == mhc.PRE_GENERIC         # fp32 storage
-    assert mhc.mhc_pre_path_for(16384, 8, 4096, 1) == mhc.PRE_GENERIC         # n = 8
+    assert mhc.mhc_pre_path_for(8192, 8, 4096, 1) == mhc.PRE_TWO_PASS_TC      # n = 8
+    for d in (6144, 7168, 8192):                                             # large d at n = 4
+        assert mhc.mhc_pre_path_for(16384, 4, d, 1) == mhc.PRE_TWO_PASS_TC, d
+    assert mhc.mhc_pre_path_for(100, 8, 4096, 1) == mhc.PRE_GENERIC           # x_in too small for scratch
     assert mhc.mhc_pre_path_for(16384, 4, 4100, 1) == mhc.PRE_GENERIC         # d % 64 != 0
     assert mhc.mhc_pre_path_for(16384, 2, 256, 1) == mhc.PRE_GENERIC          # n*d < 1024
 
