@@ -34,6 +34,11 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                  :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
+// A bf16 pair packed in a 32-bit word as an fp32 pair (element 0 first).
+__device__ __forceinline__ float2 bf16x2_to_f32x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
 // Unpack / pack a 16-byte vector of VEC elements to / from fp32.
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {

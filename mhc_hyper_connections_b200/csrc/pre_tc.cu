@@ -385,9 +385,9 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         int g = 0;
         for (int k = 0; k < my_tiles; ++k) {
-            float sv[8];                          // eight independent FMA chains
+            float2 sv[4];                         // eight independent FMA chains, in pairs
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sv[e] = 0.f;
+            for (int e = 0; e < 4; ++e) sv[e] = make_float2(0.f, 0.f);
             bool ok = true;
             for (int al = 0; al < ka; al += SA, ++g) {
                 const int na = ka - al < SA ? ka - al : SA;
@@ -403,10 +403,12 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                             w[kk] = *reinterpret_cast<const uint4*>(xs + a * (NT * 128) + (((half * 4 + kk) ^ (row & 7)) << 4));
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            float f[8];
-                            Vec16<__nv_bfloat16>::unpack(w[kk], f);
+                            const uint32_t ww[4] = {w[kk].x, w[kk].y, w[kk].z, w[kk].w};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) sv[e] = fmaf(f[e], f[e], sv[e]);
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = bf16x2_to_f32x2(ww[e]);
+                                sv[e] = __ffma2_rn(f, f, sv[e]);
+                            }
                         }
                     }
                 }
@@ -414,7 +416,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                 if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
             }
             if (!ok) break;
-            float ss = ((sv[0] + sv[1]) + (sv[2] + sv[3])) + ((sv[4] + sv[5]) + (sv[6] + sv[7]));
+            float ss = ((sv[0].x + sv[0].y) + (sv[1].x + sv[1].y)) + ((sv[2].x + sv[2].y) + (sv[3].x + sv[3].y));
             ss += __shfl_xor_sync(0xffffffffu, ss, 16);
             // accumulators of tile k: sum the issuers' partial projections
             const int b = k % NACC, ub = k / NACC;
@@ -614,17 +616,19 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
                     if (tt[u] < nt) {
                         const float4 h4 = *reinterpret_cast<const float4*>(hs + tt[u] * 4);
                         const float hv[4] = {h4.x, h4.y, h4.z, h4.w};
-                        float acc[8];
+                        float2 acc[4];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                        for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int i = 0; i < N; ++i) {
-                            float f[8];
-                            Vec16<__nv_bfloat16>::unpack(xv[u][i], f);
+                            const float2 h2 = make_float2(hv[i], hv[i]);
+                            const uint32_t ww[4] = {xv[u][i].x, xv[u][i].y, xv[u][i].z, xv[u][i].w};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) acc[e] = fmaf(hv[i], f[e], acc[e]);
+                            for (int e = 0; e < 4; ++e) acc[e] = __ffma2_rn(h2, bf16x2_to_f32x2(ww[e]), acc[e]);
                         }
-                        st_v4(ob + (tt[u] * d + cc[u] * 8), Vec16<__nv_bfloat16>::pack(acc));
+                        st_v4(ob + (tt[u] * d + cc[u] * 8),
+                              make_uint4(pack_bf16x2(acc[0].x, acc[0].y), pack_bf16x2(acc[1].x, acc[1].y),
+                                         pack_bf16x2(acc[2].x, acc[2].y), pack_bf16x2(acc[3].x, acc[3].y)));
                     }
                 }
                 if (t >= nt) break;

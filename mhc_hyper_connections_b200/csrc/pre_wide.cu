@@ -11,13 +11,14 @@
 //      phi_lo = bf16(phi - phi_hi) (16 significant bits, above the TF32 the mixed-
 //      precision table asks for), K-major with the 128-byte swizzle.  It is written into
 //      the x_in buffer, which holds nothing else until launch 3 writes x_in.
-//   2. projection: clusters of C = 8 CTAs split K = n d; a cluster takes 256-token tiles.
+//   2. projection: clusters of C = 4 CTAs split K = n d; a cluster takes 256-token tiles
+//      (4-CTA clusters fill the GPU in one wave of tiles at the n = 8 workload).
 //      Per 64-channel atom a stage holds the tile's X (one 32 KB TMA box) and the atom of
 //      packed phi (one bulk copy, served from L2).  Two warps issue tcgen05.mma
 //      (M = 128 tokens, N = 2 MH, K = 16), one per half of the tile, into TMEM; four warps
 //      add the tokens' squares.  Each CTA writes its partial projection and sum of squares
 //      of every token to a scratch block in the x_in buffer; the owner CTA of a token
-//      (32 tokens each) adds the 8 partials in a fixed order, applies 1/r and forms H.
+//      (64 tokens each) adds the 4 partials in a fixed order, applies 1/r and forms H.
 //   3. read map: x_in = sum_i H_pre[i] X[i, :], streaming X from HBM a second time.
 //
 // X crosses HBM twice here; streaming phi instead against tiles small enough to re-read
@@ -39,7 +40,7 @@ __device__ unsigned int g_pre_wide_status;
 
 namespace wide {
 
-constexpr int C = 8;               // CTAs per cluster (K split)
+constexpr int C = 4;               // CTAs per cluster (K split)
 constexpr int TT = 256;            // tokens per tile
 constexpr int HALF = 128;          // MMA M
 constexpr int TPO = TT / C;        // tokens owned per CTA and tile
@@ -51,7 +52,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int X_STAGE = TT * 128;  // one atom of a 256-token tile
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
-static_assert(TPO == 32, "one owner lane per owned token");
+static_assert(TPO % 32 == 0, "the owner warp takes TPO / 32 tokens per lane");
 
 template <int N>
 struct Cfg {
@@ -345,40 +346,46 @@ wide_proj_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __res
             }
         }
     } else if (warp == 3) {
-        // owner: tokens rank * 32 + lane of every tile; adds the C partial records in order
+        // owner: tokens rank * TPO + lane + 32 j of every tile; adds the C partial records of
+        // a token in source order
         for (int k = 0; k < my_tiles; ++k) {
             const int sl = k % NS, us = k / NS;
             if (!wait.template operator()<true>(bar(B_PFULL + sl), us & 1, E_PFULL)) break;
             const int tile = cid + k * ncl;
-            const int t = (int)rank * TPO + lane;
-            const float* rec = scratch + ((int64_t)tile * TT + t) * C * W;
-            float hv[M];
-            float ssum = 0.f;
-#pragma unroll
-            for (int j = 0; j < M; ++j) hv[j] = 0.f;
 #pragma unroll 1
-            for (int src = 0; src < C; ++src) {
-                const float* r = rec + src * W;
+            for (int j32 = 0; j32 < TPO / 32; ++j32) {
+                const int t = (int)rank * TPO + j32 * 32 + lane;
+                const float* rec = scratch + ((int64_t)tile * TT + t) * C * W;
+                float hv[M];
+                float ssum = 0.f;
 #pragma unroll
-                for (int j = 0; j < M; ++j) hv[j] += __ldcg(r + j);
-                ssum += __ldcg(r + M);
-            }
-            __syncwarp();
-            if (lane < C) mbar_arrive_remote(mapa(bar(B_PEMPTY + sl), (uint32_t)lane));
-            const int64_t tok = (int64_t)tile * TT + t;
-            const float inv_r = 1.0f / sqrtf(ssum / (float)(N * d) + eps);
+                for (int j = 0; j < M; ++j) hv[j] = 0.f;
+#pragma unroll 1
+                for (int src = 0; src < C; ++src) {
+                    const float* r = rec + src * W;
 #pragma unroll
-            for (int j = 0; j < M; ++j) hv[j] *= inv_r;
-            if (tok < T) {
-                if (h_out != nullptr) {
-#pragma unroll
-                    for (int j = 0; j < M; ++j) h_out[tok * M + j] = hv[j];
+                    for (int j = 0; j < M; ++j) hv[j] += __ldcg(r + j);
+                    ssum += __ldcg(r + M);
                 }
-                float out[M];
-                if (hc) token_maps_hc<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, out);
-                else token_maps<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+                if (j32 == TPO / 32 - 1) {   // every record of this tile has been read
+                    __syncwarp();
+                    if (lane < C) mbar_arrive_remote(mapa(bar(B_PEMPTY + sl), (uint32_t)lane));
+                }
+                const int64_t tok = (int64_t)tile * TT + t;
+                const float inv_r = 1.0f / sqrtf(ssum / (float)(N * d) + eps);
 #pragma unroll
-                for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
+                for (int j = 0; j < M; ++j) hv[j] *= inv_r;
+                if (tok < T) {
+                    if (h_out != nullptr) {
+#pragma unroll
+                        for (int j = 0; j < M; ++j) h_out[tok * M + j] = hv[j];
+                    }
+                    float out[M];
+                    if (hc) token_maps_hc<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, out);
+                    else token_maps<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+#pragma unroll
+                    for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
+                }
             }
         }
     }

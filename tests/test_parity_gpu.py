@@ -227,7 +227,8 @@ def test_auto_path_on_b200_shapes_is_tensor_core():
         assert mhc.mhc_pre_path_for(16384, 4, d, 1) == mhc.PRE_TWO_PASS_TC, d
     assert mhc.mhc_pre_path_for(100, 8, 4096, 1) == mhc.PRE_GENERIC           # x_in too small for scratch
     assert mhc.mhc_pre_path_for(16384, 4, 4100, 1) == mhc.PRE_GENERIC         # d % 64 != 0
-    assert mhc.mhc_pre_path_for(16384, 2, 256, 1) == mhc.PRE_GENERIC          # n*d < 1024
+    assert mhc.mhc_pre_path_for(16384, 2, 256, 1) == mhc.PRE_TWO_PASS_TC      # n*d = 512
+    assert mhc.mhc_pre_path_for(16384, 1, 192, 1) == mhc.PRE_GENERIC          # n*d < 256
 
 
 def test_device_status_clean_after_runs():
