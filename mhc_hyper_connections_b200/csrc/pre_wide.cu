@@ -13,8 +13,9 @@
 //      the x_in buffer, which holds nothing else until launch 3 writes x_in.
 //   2. projection: clusters of C = 4 CTAs split K = n d; a cluster takes 256-token tiles
 //      (4-CTA clusters fill the GPU in one wave of tiles at the n = 8 workload).
-//      Per 64-channel atom a stage holds the tile's X (one 32 KB TMA box) and the atom of
-//      packed phi (one bulk copy, served from L2).  Two warps issue tcgen05.mma
+//      A stage holds two 64-channel atoms: the tile's X (one 64 KB TMA box) and those atoms
+//      of packed phi (one bulk copy, served from L2) -- large boxes, since one SM's TMA
+//      unit retires only a few boxes per microsecond.  Two warps issue tcgen05.mma
 //      (M = 128 tokens, N = 2 MH, K = 16), one per half of the tile, into TMEM; four warps
 //      add the tokens' squares.  Each CTA writes its partial projection and sum of squares
 //      of every token to a scratch block in the x_in buffer; the owner CTA of a token
@@ -50,6 +51,7 @@ constexpr int NWARPS = 8;          // 0 TMA, 1-2 MMA, 3 owner, 4-7 squares + epi
 constexpr int THREADS = NWARPS * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int X_STAGE = TT * 128;  // one atom of a 256-token tile
+constexpr int SW = 2;              // atoms per stage (one 64 KB box of X, one copy of phi)
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
 static_assert(TPO % 32 == 0, "the owner warp takes TPO / 32 tokens per lane");
@@ -61,7 +63,7 @@ struct Cfg {
     static constexpr int NB = 2 * MH;                      // MMA N: [hi | lo]
     static constexpr int PHI_ATOM = NB / 8 * 1024;         // bytes of one packed atom
     static constexpr int W = ((MH > M + 1 ? MH : M + 1) + 3) / 4 * 4;   // floats per partial record
-    static constexpr int STAGE = X_STAGE + PHI_ATOM;
+    static constexpr int STAGE = SW * (X_STAGE + PHI_ATOM);
     static constexpr int NACCB = TMEM_COLS / (2 * NB) >= 2 ? 2 : 1;     // accumulator buffers
     static_assert(NB <= 256 && NB % 16 == 0, "MMA N for M = 128");
     static_assert(2 * NB <= TMEM_COLS, "both halves fit TMEM");
@@ -101,6 +103,10 @@ struct Waiter {
             }
         }
     }
+};
+
+struct WMaps {
+    CUtensorMap box[SW];           // box[j]: j + 1 atoms of a 256-token tile
 };
 
 __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
@@ -153,7 +159,7 @@ wide_pack_kernel(const float* __restrict__ phi, int ka_total, uint8_t* __restric
 // ---------------------------------------------------------------- 2. projection
 template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
-wide_proj_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ packed,
+wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__ packed,
                  float* __restrict__ scratch, const float* __restrict__ b_pre,
                  const float* __restrict__ b_post, const float* __restrict__ b_res, float a_pre,
                  float a_post, float a_res, int T, int d, float eps, int t_max,
@@ -208,20 +214,23 @@ wide_proj_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __res
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // producer: stage g = (tile g / ka, atom g % ka): the X box and the packed phi atom
+        // producer: stage g = (tile g / spt, atoms from al = (g % spt) * SW): one X box of
+        // na atoms and one copy of their packed phi
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" :: "l"(&map_x) : "memory");
-            const int total = my_tiles * ka;
+            asm volatile("prefetch.tensormap [%0];" :: "l"(&maps.box[SW - 1]) : "memory");
+            const int spt = (ka + SW - 1) / SW;
+            const int total = my_tiles * spt;
             int g = 0;
             for (; g < total; ++g) {
-                const int k = g / ka, al = g - k * ka;
+                const int k = g / spt, al = (g - k * spt) * SW;
+                const int na = ka - al < SW ? ka - al : SW;
                 const int s = g % nstage, u = g / nstage;
                 if (!wait(bar(B_EMPTY + s), (u & 1) ^ 1, E_EMPTY)) break;
                 const uint32_t st = base + (uint32_t)s * Cf::STAGE;
-                mbar_arrive_tx(bar(B_FULL + s), (uint32_t)Cf::STAGE);
-                tma_load_3d(st, &map_x, bar(B_FULL + s), 0, (cid + k * ncl) * TT, a_lo + al);
-                bulk_g2s(st + X_STAGE, packed + (int64_t)(a_lo + al) * Cf::PHI_ATOM, (uint32_t)Cf::PHI_ATOM,
-                         bar(B_FULL + s));
+                mbar_arrive_tx(bar(B_FULL + s), (uint32_t)(na * (X_STAGE + Cf::PHI_ATOM)));
+                tma_load_3d(st, &maps.box[na - 1], bar(B_FULL + s), 0, (cid + k * ncl) * TT, a_lo + al);
+                bulk_g2s(st + SW * X_STAGE, packed + (int64_t)(a_lo + al) * Cf::PHI_ATOM,
+                         (uint32_t)(na * Cf::PHI_ATOM), bar(B_FULL + s));
             }
             for (int j = g - 1; j >= 0 && j >= g - nstage; --j)
                 drain(bar(B_FULL + j % nstage), (j / nstage) & 1, E_DRAIN, false);
@@ -239,17 +248,20 @@ wide_proj_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __res
                 if (!wait(bar(B_ACCE + b), (ub & 1) ^ 1, E_ACCE)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)((b * 2 + h) * NB);
-                for (int al = 0; al < ka; ++al, ++g) {
+                for (int al = 0; al < ka; al += SW, ++g) {
+                    const int na = ka - al < SW ? ka - al : SW;
                     const int s = g % nstage, u = g / nstage;
                     if (!wait(bar(B_FULL + s), u & 1, E_FULL)) { stop = true; break; }
                     tc_fence_after();
                     const uint32_t st = base + (uint32_t)s * Cf::STAGE;
-                    const uint64_t ad = sw128_desc(st + (uint32_t)h * (HALF * 128));
-                    const uint64_t bd = sw128_desc(st + X_STAGE);
-                    mma_bf16(d_tmem, ad, bd, IDESC, al > 0 ? 1u : 0u);
-                    mma_bf16(d_tmem, ad + 2, bd + 2, IDESC, 1);
-                    mma_bf16(d_tmem, ad + 4, bd + 4, IDESC, 1);
-                    mma_bf16(d_tmem, ad + 6, bd + 6, IDESC, 1);
+                    for (int j = 0; j < na; ++j) {
+                        const uint64_t ad = sw128_desc(st + (uint32_t)(j * X_STAGE + h * (HALF * 128)));
+                        const uint64_t bd = sw128_desc(st + (uint32_t)(SW * X_STAGE + j * Cf::PHI_ATOM));
+                        mma_bf16(d_tmem, ad, bd, IDESC, (al > 0 || j > 0) ? 1u : 0u);
+                        mma_bf16(d_tmem, ad + 2, bd + 2, IDESC, 1);
+                        mma_bf16(d_tmem, ad + 4, bd + 4, IDESC, 1);
+                        mma_bf16(d_tmem, ad + 6, bd + 6, IDESC, 1);
+                    }
                     issued = 1;
                     mma_commit(bar(B_EMPTY + s));
                 }
@@ -270,33 +282,40 @@ wide_proj_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __res
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         int g = 0;
         for (int k = 0; k < my_tiles; ++k) {
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            float2 s0[4], s1[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) s0[x] = s1[x] = make_float2(0.f, 0.f);
             bool ok = true;
-            for (int al = 0; al < ka; ++al, ++g) {
+            for (int al = 0; al < ka; al += SW, ++g) {
+                const int na = ka - al < SW ? ka - al : SW;
                 const int s = g % nstage, u = g / nstage;
                 if (!wait(bar(B_FULL + s), u & 1, E_FULL)) { ok = false; break; }
-                const uint8_t* st = sb + (uint32_t)s * Cf::STAGE;
-                uint4 w0[8], w1[8];
+                for (int j = 0; j < na; ++j) {
+                    const uint8_t* st = sb + (uint32_t)s * Cf::STAGE + (uint32_t)j * X_STAGE;
+                    uint4 w0[8], w1[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    w0[c] = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((c ^ (r0 & 7)) << 4));
-                    w1[c] = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((c ^ (r1 & 7)) << 4));
-                }
+                    for (int c = 0; c < 8; ++c) {
+                        w0[c] = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((c ^ (r0 & 7)) << 4));
+                        w1[c] = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((c ^ (r1 & 7)) << 4));
+                    }
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float f[8];
-                    Vec16<__nv_bfloat16>::unpack(w0[c], f);
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t a0[4] = {w0[c].x, w0[c].y, w0[c].z, w0[c].w};
+                        const uint32_t a1[4] = {w1[c].x, w1[c].y, w1[c].z, w1[c].w};
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) s0[x & 3] = fmaf(f[x], f[x], s0[x & 3]);
-                    Vec16<__nv_bfloat16>::unpack(w1[c], f);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) s1[x & 3] = fmaf(f[x], f[x], s1[x & 3]);
+                        for (int x = 0; x < 4; ++x) {
+                            const float2 f0 = bf16x2_to_f32x2(a0[x]), f1 = bf16x2_to_f32x2(a1[x]);
+                            s0[x] = __ffma2_rn(f0, f0, s0[x]);
+                            s1[x] = __ffma2_rn(f1, f1, s1[x]);
+                        }
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_EMPTY + s));
             }
             if (!ok) break;
-            const float ss[2] = {(s0[0] + s0[1]) + (s0[2] + s0[3]), (s1[0] + s1[1]) + (s1[2] + s1[3])};
+            const float ss[2] = {((s0[0].x + s0[0].y) + (s0[1].x + s0[1].y)) + ((s0[2].x + s0[2].y) + (s0[3].x + s0[3].y)),
+                                 ((s1[0].x + s1[0].y) + (s1[1].x + s1[1].y)) + ((s1[2].x + s1[2].y) + (s1[3].x + s1[3].y))};
             const int b = k % NACCB, ub = k / NACCB;
             if (!wait(bar(B_ACCF + b), ub & 1, E_ACCF)) break;
             tc_fence_after();
@@ -567,18 +586,21 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
-        // X viewed as 3-D: (element within a 64-channel atom, token, atom); box (64, 256, 1)
-        CUtensorMap map;
+        // X viewed as 3-D: (element within a 64-channel atom, token, atom); box j: (64, 256,
+        // j + 1), stored atom-major
+        WMaps maps;
         const cuuint64_t dims[3] = {64, (cuuint64_t)a.T, (cuuint64_t)ka_total};
         const cuuint64_t strides[2] = {(cuuint64_t)N * a.d * 2, 128};
-        const cuuint32_t box[3] = {64, (cuuint32_t)TT, 1};
         const cuuint32_t estr[3] = {1, 1, 1};
         auto enc = encode_fn();
         if (!enc) return cudaErrorNotSupported;
-        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+        for (int j = 0; j < SW; ++j) {
+            const cuuint32_t box[3] = {64, (cuuint32_t)TT, (cuuint32_t)(j + 1)};
+            if (enc(&maps.box[j], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
         const int num_tiles = (int)((a.T + TT - 1) / TT);
         const int ncl = num_tiles < p.max_clusters ? num_tiles : p.max_clusters;
         cudaLaunchConfig_t cfg = {};
@@ -593,7 +615,7 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p) {
         at[0].val.clusterDim.z = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, wide_proj_kernel<N>, map, static_cast<const uint8_t*>(packed), scratch,
+        e = cudaLaunchKernelEx(&cfg, wide_proj_kernel<N>, maps, static_cast<const uint8_t*>(packed), scratch,
                                a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps,
                                a.t_max, a.H, a.h_out, ka_total, p.nstage, a.hc ? 1 : 0, g_wait_ns);
         if (e != cudaSuccess) return e;

@@ -108,7 +108,7 @@ SHAPES = [  # (T, n, d, dtype): ragged token tails, odd d, every n
     # two-pass tensor-core path: n = 5..8, and d past the cluster kernel's shared memory
     (2000, 8, 4096, "bf16"), (2100, 7, 2048, "bf16"), (1500, 6, 1536, "bf16"),
     (2100, 5, 1024, "bf16"), (400, 4, 8192, "bf16"), (350, 4, 7168, "bf16"), (300, 4, 6144, "bf16"),
-    (1300, 4, 2048, "bf16"), (700, 3, 1024, "bf16"),
+    (1300, 4, 2048, "bf16"), (700, 3, 1024, "bf16"), (900, 5, 1088, "bf16"),
 ]
 
 
