@@ -207,6 +207,9 @@ size_t mhc_backward_workspace_bytes(int64_t T, int n, int d);
  * Limits : n <= 4 (MHC_ERR_UNSUPPORTED above); X, F_out, dX_out, dx_in, dX and dF_out
  *          16-byte aligned with d * sizeof(element) a multiple of 16 (else MHC_ERR_ALIGN).
  *          No output may overlap an input or another output (MHC_ERR_ALIAS).
+ * Kernels: bf16 with d a multiple of 64 runs the products phi G (for dX) and X^T G (dphi)
+ *          on the tensor cores with G and phi split into bf16 hi + lo parts (16 significant
+ *          bits each, fp32 accumulation); other shapes and fp32 run them on CUDA cores.
  */
 mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, const float* b_pre,
                         const float* b_post, const float* b_res, float alpha_pre, float alpha_post,
@@ -275,8 +278,9 @@ mhc_status mhc_amax_gain(const float* H_layers, int L, int64_t T, int n, float* 
  * mhc_device_status -- read and clear the device-side status words of the tensor-core
  * kernels.  Their waits between warps and between the CTAs of a cluster are bounded in
  * time (1 s each); a wait that expires makes the kernel stop early, leaving its outputs
- * incomplete, and sets a bit here naming the wait.  *code = 0 means every wait of every
- * launch since the last read completed.  Blocks until prior work on the legacy default
+ * incomplete, and sets a bit here naming the wait: bits 0-15 the cluster pre kernel, 16-23
+ * the two-pass pre kernels, 24-31 the tensor-core dX / dphi step of mhc_backward.  *code = 0
+ * means every wait of every launch since the last read completed.  Blocks until prior work on the legacy default
  * stream (and streams that synchronise with it) has finished.  No counterpart on the
  * pages: this is the library's failure report.
  */

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(TOK_THREADS)
 bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const float* __restrict__ h,
                  const float* __restrict__ b_res, float a_pre, float a_post, float a_res,
                  int64_t Tn, int K, float eps, int t_max, float* __restrict__ dl,
-                 float* __restrict__ G, float* __restrict__ beta) {
+                 float* __restrict__ G, float* __restrict__ beta, unsigned char* __restrict__ rec) {
     constexpr int M = N * N + 2 * N, NR = red_len(N);
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= Tn) return;
@@ -228,16 +228,58 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         for (int j = 0; j < N; ++j) out[N + i * N + j] = gM[i][j] * M0[i][j];
     // g = alpha * dl; G = g / r; beta = (g . h) / (K r^2)
     const float inv_r = 1.0f / sqrtf(Rt[0] / (float)K + eps);
-    float gh = 0.f;
+    float gh = 0.f, Gv[M];
 #pragma unroll
     for (int j = 0; j < M; ++j) {
         const float a = j < N ? a_pre : (j < N + N * N ? a_res : a_post);
         const float g = a * out[j];
         gh = fmaf(g, hh[j], gh);
         dl[t * M + j] = out[j];
-        G[t * M + j] = g * inv_r;
+        Gv[j] = g * inv_r;
     }
-    beta[t] = gh * inv_r * inv_r / (float)K;
+    const float bt = gh * inv_r * inv_r / (float)K;
+    if (rec == nullptr) {
+#pragma unroll
+        for (int j = 0; j < M; ++j) G[t * M + j] = Gv[j];
+        beta[t] = bt;
+        return;
+    }
+    // the tensor-core step's record (launch.cuh): [G_hi | G_lo], [G_hi | 0], coefficients
+    uint4* r4 = reinterpret_cast<uint4*>(rec + t * BWD_REC_BYTES);
+    uint32_t w[32];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        __nv_bfloat16 hv[2], lv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = 2 * e + u;
+            const float v = j < M ? Gv[j] : 0.f;
+            hv[u] = __float2bfloat16(v);
+            lv[u] = __float2bfloat16(v - __bfloat162float(hv[u]));
+        }
+        w[e] = (uint32_t)__bfloat16_as_ushort(hv[0]) | ((uint32_t)__bfloat16_as_ushort(hv[1]) << 16);
+        w[16 + e] = (uint32_t)__bfloat16_as_ushort(lv[0]) | ((uint32_t)__bfloat16_as_ushort(lv[1]) << 16);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        r4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        r4[8 + e] = e < 4 ? make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]) : make_uint4(0, 0, 0, 0);
+    }
+    float4* c4 = reinterpret_cast<float4*>(rec + t * BWD_REC_BYTES + 256);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float cf[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cf[q] = 0.f;
+        if (i < N) {
+            cf[0] = H[t * M + i];
+#pragma unroll
+            for (int p = 0; p < N; ++p) cf[1 + p] = H[t * M + N + p * N + i];
+            cf[5] = -bt;
+        }
+        c4[2 * i] = make_float4(cf[0], cf[1], cf[2], cf[3]);
+        c4[2 * i + 1] = make_float4(cf[4], cf[5], cf[6], cf[7]);
+    }
 }
 
 // ---------------------------------------------------------------- K3
@@ -404,9 +446,13 @@ cudaError_t launch_n(const BwdArgs& a, const BwdLayout& L) {
         bwd_reduce_kernel<N, T><<<(unsigned)blocks, RED_THREADS, 0, a.stream>>>(
             X, static_cast<const T*>(a.F), dY, dxi, a.H, Tn, d, R, static_cast<T*>(a.dF_out));
     }
+    unsigned char* rec = L.tc ? reinterpret_cast<unsigned char*>(ws + L.off_rec) : nullptr;
     bwd_token_kernel<N><<<(unsigned)((Tn + TOK_THREADS - 1) / TOK_THREADS), TOK_THREADS, 0, a.stream>>>(
-        R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res, Tn, K, a.eps, a.t_max, dl, G, beta);
-    {
+        R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res, Tn, K, a.eps, a.t_max, dl, G, beta, rec);
+    if (L.tc) {
+        e = launch_bwd_tc(a, rec, part, L.groups, L.tokens_per_group);
+        if (e != cudaSuccess) return e;
+    } else {
         const int cs = dx_slice(N);
         dim3 grid((unsigned)((d + cs - 1) / cs), (unsigned)L.groups);
         bwd_dx_dphi_kernel<N, T><<<grid, DX_THREADS, 0, a.stream>>>(
@@ -436,31 +482,47 @@ cudaError_t dispatch(const BwdArgs& a, const BwdLayout& L) {
 
 }  // namespace
 
-BwdLayout backward_layout(int64_t T, int n, int d) {
+BwdLayout backward_layout(int64_t T, int n, int d, bool tc) {
     BwdLayout L{};
     const int64_t m = (int64_t)n * n + 2 * n, K = (int64_t)n * d;
-    const int64_t slices = (d + dx_slice(n) - 1) / dx_slice(n);
-    // about 1024 CTAs in K3, each group at least 32 tokens
-    int64_t groups = (1024 + slices - 1) / slices;
-    const int64_t max_groups = (T + TB - 1) / TB;
-    if (groups > max_groups) groups = max_groups;
-    if (groups < 1) groups = 1;
-    L.groups = (int)groups;
-    L.tokens_per_group = (T + groups - 1) / groups;
+    L.tc = tc && d % 64 == 0 && d >= 64;
+    if (L.tc) {
+        L.groups = bwd_tc_groups(T, d, BWD_TC_SMS);
+        L.tokens_per_group = bwd_tc_tokens_per_group(T, L.groups);
+    } else {
+        const int64_t slices = (d + dx_slice(n) - 1) / dx_slice(n);
+        // about 1024 CTAs in K3, each group at least 32 tokens
+        int64_t groups = (1024 + slices - 1) / slices;
+        const int64_t max_groups = (T + TB - 1) / TB;
+        if (groups > max_groups) groups = max_groups;
+        if (groups < 1) groups = 1;
+        L.groups = (int)groups;
+        L.tokens_per_group = (T + groups - 1) / groups;
+    }
     auto up = [](int64_t x) { return (x + 63) / 64 * 64; };   // 256-byte aligned regions
     int64_t off = 0;
     L.off_R = off;      off += up(T * red_len(n));
     L.off_dl = off;     off += up(T * m);
-    L.off_G = off;      off += up(T * m);
-    L.off_beta = off;   off += up(T);
-    L.off_part = off;   off += up(groups * K * m);
+    if (L.tc) {
+        L.off_rec = off; off += up(T * (BWD_REC_BYTES / 4));
+    } else {
+        L.off_G = off;      off += up(T * m);
+        L.off_beta = off;   off += up(T);
+    }
+    L.off_part = off;   off += up((int64_t)L.groups * K * m);
     L.off_colsum = off; off += up(2 * m);
     L.floats = off;
     return L;
 }
 
+int64_t backward_workspace_floats(int64_t T, int n, int d) {
+    const int64_t a = backward_layout(T, n, d, false).floats, b = backward_layout(T, n, d, true).floats;
+    return a > b ? a : b;
+}
+
 cudaError_t launch_backward(const BwdArgs& a) {
-    const BwdLayout L = backward_layout(a.T, a.n, a.d);
+    const bool tc = bwd_tc_shape_ok(a.T, a.n, a.d, a.dt) && bwd_tc_device_ok(a.n);
+    const BwdLayout L = backward_layout(a.T, a.n, a.d, tc);
     return a.dt == BF16 ? dispatch<__nv_bfloat16>(a, L) : dispatch<float>(a, L);
 }
 

@@ -98,13 +98,30 @@ struct BwdArgs {
     cudaStream_t stream;
 };
 
-// Workspace regions, in floats from the (256-byte aligned) workspace base.
+// Workspace regions, in floats from the (256-byte aligned) workspace base.  The tensor-core
+// dX / dphi step (tc) reads per-token records instead of G and beta.
 struct BwdLayout {
-    int64_t off_R, off_dl, off_G, off_beta, off_part, off_colsum, floats;
+    int64_t off_R, off_dl, off_G, off_beta, off_rec, off_part, off_colsum, floats;
     int groups;                  // token groups of the dX / dphi kernel
     int64_t tokens_per_group;
+    bool tc;
 };
-BwdLayout backward_layout(int64_t T, int n, int d);
+BwdLayout backward_layout(int64_t T, int n, int d, bool tc);
+// workspace the backward needs whichever dX / dphi kernel it takes, in floats
+int64_t backward_workspace_floats(int64_t T, int n, int d);
+
+// Tensor-core dX / dphi step (backward_tc.cu): bf16, n <= 4, d a multiple of 64.  It reads one
+// record of BWD_REC_BYTES per token, written by the token kernel: row 0 = [G_hi | G_lo], row 1
+// = [G_hi | 0] (bf16, 32 each, zero past m), row 2 = per stream i < 4 the fp32 coefficients
+// {H_pre[i], H_res[0..3][i], -beta, 0, 0} (zero past n).
+constexpr int BWD_REC_BYTES = 384;
+constexpr int BWD_TC_SMS = 148;   // groups are sized for this many SMs (results do not depend on the device)
+bool bwd_tc_shape_ok(int64_t T, int n, int d, DType dt);
+bool bwd_tc_device_ok(int n);
+int bwd_tc_groups(int64_t T, int d, int sm_count);
+int64_t bwd_tc_tokens_per_group(int64_t T, int groups);
+cudaError_t launch_bwd_tc(const BwdArgs& a, const void* rec, float* part, int groups, int64_t tpg);
+cudaError_t bwd_tc_status(unsigned* out, bool clear);
 
 // Amax Gain Magnitude of composite residual maps (diagnostics.cu).
 cudaError_t launch_amax_gain(const float* Hs, int L, int64_t T, int n, float* gain, cudaStream_t s);

@@ -213,7 +213,7 @@ mhc_status mhc_pre_train(const void* X, const float* phi, const float* b_pre, co
 
 size_t mhc_backward_workspace_bytes(int64_t T, int n, int d) {
     if (check_shape(T, n, d, MHC_F32) != MHC_OK || n > 4) return 0;
-    return (size_t)backward_layout(T, n, d).floats * 4;
+    return (size_t)backward_workspace_floats(T, n, d) * 4;
 }
 
 mhc_status mhc_backward(const void* X, const void* F_out, const float* phi, const float* b_pre,
@@ -348,11 +348,12 @@ mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us) {
 
 mhc_status mhc_device_status(uint32_t* code) {
     if (!code) return MHC_ERR_NULL;
-    unsigned v = 0, w = 0;
+    unsigned v = 0, w = 0, b = 0;
     cudaError_t e = pre_tc_status(&v, true);
     if (e == cudaSuccess) e = pre_wide_status(&w, true);
+    if (e == cudaSuccess) e = bwd_tc_status(&b, true);
     if (e != cudaSuccess) return cuda_fail(e, "mhc_device_status");
-    *code = v | (w << 16);
+    *code = v | (w << 16) | (b << 24);
     return MHC_OK;
 }
 

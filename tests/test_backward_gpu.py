@@ -118,8 +118,13 @@ def test_bf16_d1024_full():
 
 
 @pytest.mark.parametrize("T,n,d,dt", [(1, 1, 8, "bf16"), (33, 2, 24, "f32"), (100, 3, 136, "bf16"),
-                                      (37, 4, 64, "bf16"), (300, 1, 1024, "bf16"), (65, 3, 12, "f32")])
+                                      (37, 4, 64, "bf16"), (300, 1, 1024, "bf16"), (65, 3, 12, "f32"),
+                                      (129, 3, 192, "bf16"), (1000, 2, 640, "bf16"), (64, 4, 128, "bf16"),
+                                      (200, 4, 4096, "bf16"), (1, 2, 64, "bf16"), (777, 1, 128, "bf16")])
 def test_shapes(T, n, d, dt):
+    """Ragged shapes on both dX / dphi kernels: bf16 with d a multiple of 64 takes the
+    tensor-core step (token tails inside a stage, groups that end mid-tensor or hold no
+    tokens, odd n with a placeholder stream), the rest the CUDA-core step."""
     w = wl.make_inputs(T=T, n=n, d=d, dtype=dt, seed=T * 7 + n * 3 + d, alpha=0.3)
     dY, dx = _upstream(w, T + d)
     check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"T{T} n{n} d{d} {dt}")
@@ -134,6 +139,15 @@ def test_sinkhorn_depths(t_max, n):
     w = dataclasses.replace(w, t_max=t_max)
     dY, dx = _upstream(w, 600 + t_max)
     check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"t_max {t_max} n {n}")
+
+
+@pytest.mark.parametrize("t_max", [0, 1, 41])
+def test_sinkhorn_depths_tensor_core_step(t_max):
+    """The same depths with d a multiple of 64, so the tensor-core dX / dphi step runs."""
+    w = wl.make_inputs(T=150, n=4, d=128, dtype="bf16", seed=700 + t_max, alpha=0.3)
+    w = dataclasses.replace(w, t_max=t_max)
+    dY, dx = _upstream(w, 800 + t_max)
+    check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"t_max {t_max} tensor-core step")
 
 
 def test_headline_size_sampled_and_additive():
