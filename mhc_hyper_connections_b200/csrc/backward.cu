@@ -244,7 +244,7 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         beta[t] = bt;
         return;
     }
-    // the tensor-core step's record (launch.cuh): [G_hi | G_lo], [G_hi | 0], coefficients
+    // the tensor-core step's record (launch.cuh): [G_hi | G_lo], then the coefficients
     uint4* r4 = reinterpret_cast<uint4*>(rec + t * BWD_REC_BYTES);
     uint32_t w[32];
 #pragma unroll
@@ -261,11 +261,8 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         w[16 + e] = (uint32_t)__bfloat16_as_ushort(lv[0]) | ((uint32_t)__bfloat16_as_ushort(lv[1]) << 16);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        r4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-        r4[8 + e] = e < 4 ? make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]) : make_uint4(0, 0, 0, 0);
-    }
-    float4* c4 = reinterpret_cast<float4*>(rec + t * BWD_REC_BYTES + 256);
+    for (int e = 0; e < 8; ++e) r4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+    float4* c4 = reinterpret_cast<float4*>(rec + t * BWD_REC_BYTES + 128);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float cf[8];

@@ -10,26 +10,29 @@
 //   dphi[k][j]  = sum_t X[t][k] G_t[j]
 //
 // Both products are thin (one side is m = n^2 + 2n wide).  On tcgen05:
-//   * CTA (s, g) owns channels [64 s, 64 s + 64) of every stream and the tokens of group g.
-//     Its MMA rows are k: block b holds stream 2b in rows 0-63 and stream 2b + 1 in rows
-//     64-127 (for odd n the last block's upper half is a placeholder whose rows are unused).
-//   * phi G: A = the CTA's rows of phi, resident in TMEM as bf16 with K = 96,
-//     [phi_hi | phi_hi | phi_lo]; B = the token's record [G_hi | G_lo | G_hi], K-major in
-//     shared memory.  The sum is phi G less the phi_lo G_lo term: 16 significant bits on
-//     both sides.  D[k][t] (M = 128, N = 64 tokens) lands in TMEM, two buffers deep.
+//   * CTA (s, g) owns channels [64 s, 64 s + 64) of every stream and the tokens of group g:
+//     k rows 0-63 are stream 0 of the slice, 64-127 stream 1, and so on (for odd n a
+//     placeholder stream fills the last 64 rows; its results are not used).
+//   * phi G as D[t][k]: A = G_t as bf16 [G_hi | G_lo] (one 128-byte row of the token's
+//     record, written by the token kernel), B = the CTA's rows of phi, resident in shared
+//     memory as [phi_hi | phi_hi] and [phi_lo | 0]; the sum is phi G less the phi_lo G_lo
+//     term (16 significant bits on both sides).  A stage's 64 tokens are M: streams 0-1 go
+//     to one M = 64 accumulator in TMEM lanes 0-15 of each lane quarter, streams 2-3 to a
+//     second in lanes 16-31, so every lane of a TMEM load holds a token.
 //   * dphi: A = X^T, read by the tensor core straight from the stage's TMA tile (MN-major:
 //     64 channels in each 128-byte row, tokens down the rows); B = [G_hi | G_lo] from the
-//     same records (MN-major).  D[k][j] accumulates in TMEM over all of the group's tokens.
-//   * Eight warps form dX.  TMEM lane = row k, so a thread owns channel c of two streams; it
-//     walks the stage's tokens, reading X, dX_out and dx_in from shared memory and the
-//     token's coefficients (H_pre[i], H_res[.][i], -beta) from the record.
+//     same rows (MN-major).  D[k][j] (M = 128: two streams) accumulates in TMEM over all
+//     of the group's tokens.
+//   * Eight warps form dX: a thread owns a token, two streams and 32 channels; it reads X,
+//     dX_out and dx_in from the stage in 16-byte vectors, its token's coefficients
+//     (H_pre[i], H_res[.][i], -beta) from the record, and writes dX 8 channels at a time.
 //
 // A stage is 64 tokens: TMA boxes of the CTA's slice of X and dX_out (64 channels x 64
-// tokens x n streams), of dx_in (64 x 64) and of the 64 token records (384 B each).
-// Warp roles (320 threads): 0 TMA producer, 1 TMEM owner and MMA issuer, 2-9 phi into TMEM
-// at the start, the dX epilogue, the dphi partials at the end.  Every wait on an mbarrier is
-// bounded in time; on expiry the kernel records the wait in a status word and returns
-// after its copies and MMAs in flight have completed.
+// tokens x n streams), of dx_in (64 x 64) and of the 64 tokens' G rows.
+// Warp roles (320 threads): 0 TMA producer, 1 TMEM owner and MMA issuer, 2-9 phi into shared
+// memory at the start, the dX epilogue, the dphi partials at the end.  Every wait on an
+// mbarrier is bounded in time; on expiry the kernel records the wait in a status word and
+// returns after its copies and MMAs in flight have completed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,47 +50,62 @@ __device__ unsigned int g_bwd_tc_status;
 
 namespace bwdtc {
 
-constexpr int TT = 64;                 // tokens per stage = N of the phi G product
+constexpr int TT = 64;                 // tokens per stage = M of the phi G product
 constexpr int CW = 64;                 // channels of a CTA's slice (one 128-byte row)
 constexpr int ROW = 128;               // bytes per row of a tile
 constexpr int NBUF = 2;                // phi G accumulator buffers
+constexpr int PGN = 128;               // N of one phi G MMA: two streams of the slice
 constexpr int EPI = 8;                 // epilogue warps: two per TMEM lane quarter
 constexpr int THREADS = 32 * (2 + EPI);
 constexpr int KP16 = 6;                // K16 steps of phi G (K = 96)
-constexpr int SMEM_STAGES_MAX = 200 * 1024;
+constexpr int SMEM_LIMIT = 232448 - 512;   // dynamic shared memory, less the static part
 constexpr unsigned long long kWaitNs = 1000000000ull;    // 1 s per wait
 constexpr unsigned long long kDrainNs = 2000000000ull;   // 2 s for the drains at exit
+constexpr uint32_t kSuspendNs = 20000;  // a waiting thread sleeps up to this long per try
 
 template <int N>
 struct Cfg {
     static constexpr int M = N * N + 2 * N;
-    static constexpr int NB = (N + 1) / 2;                 // MMA row blocks of 128
+    static constexpr int NB = (N + 1) / 2;                 // stream pairs (dphi blocks, phi G halves)
+    static constexpr int NR = NB * PGN;                    // k rows of phi, placeholder rows included
+    static constexpr int PHI = 2 * NR * ROW;               // [phi_hi | phi_hi] and [phi_lo | 0] panels
     static constexpr int XB = N * TT * ROW;                // X or dX_out box
     static constexpr int DXB = TT * ROW;                   // dx_in box
-    static constexpr int GB = 3 * TT * ROW;                // token records box
+    static constexpr int GB = TT * ROW;                    // G rows of the stage's tokens
     static constexpr int STAGE = 2 * XB + DXB + GB;
-    static constexpr int NS = SMEM_STAGES_MAX / STAGE > 4 ? 4 : SMEM_STAGES_MAX / STAGE;
-    static constexpr int SMEM = NS * STAGE + 1024;         // + alignment slack
-    static constexpr int PG_COL = 0;                       // [buf][b]: TT columns each
-    static constexpr int DPHI_COL = NBUF * NB * TT;        // [b]: 64 columns each
-    static constexpr int A_COL = DPHI_COL + NB * 64;       // [b]: 48 columns each
-    static constexpr int COLS = A_COL + NB * 48;
+    static constexpr int NS_FIT = (SMEM_LIMIT - 1024 - PHI) / STAGE;
+    static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+    static constexpr int SMEM = NS * STAGE + PHI + 1024;   // + alignment slack
+    static constexpr int PG_COL = 0;                       // [buf]: PGN columns, lane base 16 per half
+    static constexpr int DPHI_COL = NBUF * PGN;            // [b]: 64 columns each
+    static constexpr int COLS = DPHI_COL + NB * 64;
     static constexpr int TMEM_COLS = COLS <= 256 ? 256 : 512;
     static_assert(M <= 32, "G_hi, G_lo fit 32 columns each");
     static_assert(NS >= 2, "at least two stages");
+    static_assert(SMEM <= SMEM_LIMIT, "shared memory");
     static_assert(COLS <= 512, "TMEM columns");
     static_assert(N <= 4, "coefficients of at most 4 streams per record");
 };
 
-// instruction descriptor, kind::f16: D fp32, A and B bf16, M = 128, N = nb
-__host__ __device__ constexpr uint32_t idesc(int nb, int a_mn, int b_mn) {
+// instruction descriptor, kind::f16: D fp32, A and B bf16, M = mm, N = nb
+__host__ __device__ constexpr uint32_t idesc(int mm, int nb, int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-           ((uint32_t)(nb >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+           ((uint32_t)(nb >> 3) << 17) | ((uint32_t)(mm >> 4) << 24);
 }
 
 enum : unsigned { E_EMPTY = 1u, E_FULL = 2u, E_PGEMPTY = 4u, E_PGFULL = 8u, E_DRAIN = 16u };
 
 using namespace ptx;
+
+// try_wait that may suspend the thread until the phase completes or `ns` pass
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
 
 struct Waiter {
     volatile int* abort_flag;
@@ -98,7 +116,7 @@ struct Waiter {
         if (mbar_try(bar, parity)) return true;
         const uint64_t t0 = gtimer();
         while (true) {
-            if (mbar_try(bar, parity)) return true;
+            if (mbar_try_sleep(bar, parity, kSuspendNs)) return true;
             if (honour_abort && *abort_flag) return false;
             if (gtimer() - t0 > limit_ns) {
                 atomicOr(&g_bwd_tc_status, code);
@@ -109,46 +127,62 @@ struct Waiter {
     }
 };
 
-__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+template <int W>
+__device__ __forceinline__ void tmem_ld_x(uint32_t taddr, uint32_t (&r)[W]);
+template <>
+__device__ __forceinline__ void tmem_ld_x<32>(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                   "=r"(r[31])
                  : "r"(taddr) : "memory");
 }
 // wait for this thread's TMEM loads; the registers are operands, so no use of them is
 // scheduled before the wait
-__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
                    "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
-                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]) :: "memory");
+                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                   "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                   "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                   "+r"(r[31]) :: "memory");
 }
-__device__ __forceinline__ float ld_bf16(const unsigned char* p) {
-    return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short*>(p)) << 16);
-}
+// bf16 pair (low, high halves of a word) to two floats
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
     return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+__device__ __forceinline__ uint32_t pack_f32x2(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 struct Maps {
     CUtensorMap x;      // X viewed as (c: d, t: T, i: n), box (64, TT, n)
     CUtensorMap dy;     // dX_out, the same view
     CUtensorMap dx;     // dx_in (c: d, t: T), box (64, TT)
-    CUtensorMap rec;    // token records (e: 64, t: T, row: 3), box (64, TT, 3)
+    CUtensorMap g;      // G rows of the token records (e: 64, t: T), box (64, TT)
 };
 
 enum : int { B_FULL = 0, B_EMPTY = 4, B_PGF = 8, B_PGE = 10, B_COUNT = 12 };
 
 template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
-bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, int T, int d, int tpg,
-              __nv_bfloat16* __restrict__ dX, float* __restrict__ part) {
+bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi,
+              const unsigned char* __restrict__ rec, int T, int d, int tpg, __nv_bfloat16* __restrict__ dX,
+              float* __restrict__ part) {
     using C = Cfg<N>;
     constexpr int M = C::M, NB = C::NB, NS = C::NS;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    unsigned char* phs = sm + NS * C::STAGE;          // phi panels: [phi_hi | phi_hi], then [phi_lo | 0]
     __shared__ __align__(8) uint64_t bars[B_COUNT];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
@@ -179,42 +213,39 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+
+    // the CTA's rows of phi as the B operand of phi G: row r is stream r / 64, channel r % 64
+    for (int r = threadIdx.x; r < C::NR; r += THREADS) {
+        const int i = r / CW, c = r % CW;
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            __nv_bfloat16 hv[2], lv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int j = 2 * e + u;
+                const float v = (j < M && i < N) ? __ldg(phi + ((int64_t)i * d + c0 + c) * M + j) : 0.f;
+                hv[u] = __float2bfloat16(v);
+                lv[u] = __float2bfloat16(v - __bfloat162float(hv[u]));
+            }
+            hw[e] = pack_bf16x2(hv[0], hv[1]);
+            lw[e] = pack_bf16x2(lv[0], lv[1]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            const uint4 hv4 = make_uint4(hw[4 * ch], hw[4 * ch + 1], hw[4 * ch + 2], hw[4 * ch + 3]);
+            *reinterpret_cast<uint4*>(phs + sw128_off(r, ch)) = hv4;
+            *reinterpret_cast<uint4*>(phs + sw128_off(r, ch + 4)) = hv4;
+            *reinterpret_cast<uint4*>(phs + C::NR * ROW + sw128_off(r, ch)) =
+                make_uint4(lw[4 * ch], lw[4 * ch + 1], lw[4 * ch + 2], lw[4 * ch + 3]);
+            *reinterpret_cast<uint4*>(phs + C::NR * ROW + sw128_off(r, ch + 4)) = make_uint4(0, 0, 0, 0);
+        }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_slot;
-
-    // phi rows into TMEM: epilogue warp (quarter q, half b) writes row 32 q + lane of block b
-    if (warp >= 2) {
-        const int q = warp & 3, b = (warp - 2) >> 2;
-        if (b < NB) {
-            const int i = 2 * b + (q >> 1), c = 32 * (q & 1) + lane;
-            __nv_bfloat16 hi[32], lo[32];
-            const __nv_bfloat16 z = __float2bfloat16(0.f);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float v = (j < M && i < N) ? __ldg(phi + ((int64_t)i * d + c0 + c) * M + j) : 0.f;
-                hi[j] = __float2bfloat16(v);
-                lo[j] = j < M ? __float2bfloat16(v - __bfloat162float(hi[j])) : z;
-            }
-            uint4 w[12];
-            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {            // K 0..31: hi; 32..63: hi; 64..95: lo
-                wp[e] = pack_bf16x2(hi[2 * e], hi[2 * e + 1]);
-                wp[16 + e] = wp[e];
-                wp[32 + e] = pack_bf16x2(lo[2 * e], lo[2 * e + 1]);
-            }
-            const uint32_t ta = tm + ((uint32_t)(32 * q) << 16) + C::A_COL + 48 * b;
-            tmem_st16(ta, *reinterpret_cast<const uint4(*)[4]>(&w[0]));
-            tmem_st16(ta + 16, *reinterpret_cast<const uint4(*)[4]>(&w[4]));
-            tmem_st16(ta + 32, *reinterpret_cast<const uint4(*)[4]>(&w[8]));
-            tmem_wait_st();
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -230,7 +261,7 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
                 tma_load_3d(base, &maps.x, full, c0, t0, 0);
                 tma_load_3d(base + C::XB, &maps.dy, full, c0, t0, 0);
                 tma_load_2d(base + 2 * C::XB, &maps.dx, full, c0, t0);
-                tma_load_3d(base + 2 * C::XB + C::DXB, &maps.rec, full, 0, t0, 0);
+                tma_load_2d(base + 2 * C::XB + C::DXB, &maps.g, full, 0, t0);
                 issued = it + 1;
             }
             // the copies of the last stages must have landed before the CTA exits
@@ -241,8 +272,9 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t ID_DPHI = idesc(64, 1, 1);   // A = X^T, B = [G_hi | G_lo], both MN-major
-            constexpr uint32_t ID_PG = idesc(TT, 0, 0);     // A = phi (TMEM), B = records, K-major
+            constexpr uint32_t ID_DPHI = idesc(128, 64, 1, 1);   // A = X^T, B = [G_hi | G_lo], MN-major
+            constexpr uint32_t ID_PG = idesc(64, PGN, 0, 0);     // A = G rows, B = phi rows, K-major
+            const uint32_t ph0 = smem_u32(phs), ph1 = ph0 + C::NR * ROW;
             int done = 0;
             for (int it = 0; it < nst; ++it) {
                 const int st = it % NS, buf = it & 1;
@@ -259,13 +291,15 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
                                  sw128_desc_mn(xs + 2 * b * TT * ROW + k * 2048, TT * ROW, 1024),
                                  sw128_desc_mn(gs + k * 2048, TT * ROW, 1024), ID_DPHI,
                                  (it > 0 || k > 0) ? 1u : 0u);
+                // phi G: pair b of streams into lanes 16 b .. 16 b + 15 of each lane quarter
 #pragma unroll
                 for (int b = 0; b < NB; ++b)
 #pragma unroll
-                    for (int k = 0; k < KP16; ++k)
-                        mma_bf16_tmem_a(tm + C::PG_COL + (buf * NB + b) * TT, tm + C::A_COL + 48 * b + 8 * k,
-                                        sw128_desc(gs + (k >> 2) * TT * ROW + (k & 3) * 32), ID_PG,
-                                        k > 0 ? 1u : 0u);
+                    for (int k = 0; k < KP16; ++k) {
+                        const uint32_t bsrc = k < 4 ? ph0 + b * PGN * ROW + 32 * k : ph1 + b * PGN * ROW + 32 * (k - 4);
+                        mma_bf16(tm + ((uint32_t)(16 * b) << 16) + C::PG_COL + buf * PGN, sw128_desc(gs + 32 * (k & 3)),
+                                 sw128_desc(bsrc), ID_PG, k > 0 ? 1u : 0u);
+                    }
                 mma_commit(bar(B_PGF + buf));
                 done = it + 1;
             }
@@ -275,54 +309,81 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- dX epilogue
+        // thread: token row tl of the stage, stream pair hp (TMEM lanes 16 hp.. of the quarter),
+        // channels [cb, cb + 32) of the slice
         const int q = warp & 3, h = (warp - 2) >> 2;
-        const int ih = q >> 1, c = 32 * (q & 1) + lane;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int tl = 16 * q + (lane & 15), hp = lane >> 4, cb = 32 * h;
+        const uint32_t tq = tm + ((uint32_t)(32 * q) << 16);
         bool ok = true;
         for (int it = 0; it < nst; ++it) {
             const int st = it % NS, buf = it & 1;
+            const int t = t_lo + it * TT + tl;
+            // the token's coefficients for the thread's two streams: H_pre[i], H_res[0..3][i], -beta
+            float cf[2][8];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int i = 2 * hp + j;
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+                if (i < N && t < t_hi) {
+                    const float4* cp = reinterpret_cast<const float4*>(rec + (int64_t)t * BWD_REC_BYTES + 128 + 32 * i);
+                    a = __ldg(cp);
+                    b = __ldg(cp + 1);
+                }
+                cf[j][0] = a.x; cf[j][1] = a.y; cf[j][2] = a.z; cf[j][3] = a.w;
+                cf[j][4] = b.x; cf[j][5] = b.y; cf[j][6] = b.z; cf[j][7] = b.w;
+            }
             if (!wait(bar(B_FULL + st), (uint32_t)(it / NS) & 1u, E_FULL) ||
                 !wait(bar(B_PGF + buf), (uint32_t)(it >> 1) & 1u, E_PGFULL)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            uint32_t pg0[32], pg1[32];
+            tmem_ld_x<32>(tq + C::PG_COL + buf * PGN + cb, pg0);            // stream 2 hp
+            tmem_ld_x<32>(tq + C::PG_COL + buf * PGN + CW + cb, pg1);       // stream 2 hp + 1
+            tmem_wait32(pg0);
+            tmem_wait32(pg1);
             const unsigned char* xs = sm + st * C::STAGE;
             const unsigned char* ys = xs + C::XB;
             const unsigned char* ds = xs + 2 * C::XB;
-            const unsigned char* cs = ds + C::DXB + 2 * TT * ROW;     // record row 2: coefficients
-            const int t0 = t_lo + it * TT;
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                const int col = h * 32 + ch * 16;
-                uint32_t pg[NB][16];
 #pragma unroll
-                for (int b = 0; b < NB; ++b) tmem_ld16_nowait(tm + lane_base + C::PG_COL + (buf * NB + b) * TT + col, pg[b]);
+            for (int cc = 0; cc < 4; ++cc) {
+                const uint32_t roff = sw128_off(tl, 4 * h + cc);
+                float dxf[8], dyf[N][8];
+                {
+                    const uint4 w = *reinterpret_cast<const uint4*>(ds + roff);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int b = 0; b < NB; ++b) tmem_wait16(pg[b]);
+                    for (int e = 0; e < 4; ++e) { dxf[2 * e] = bf_lo(ww[e]); dxf[2 * e + 1] = bf_hi(ww[e]); }
+                }
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int tl = col + u;
-                    const int t = t0 + tl;
-                    const uint32_t roff = sw128_off(tl, c >> 3) + (c & 7) * 2;
-                    const float dxv = ld_bf16(ds + roff);
-                    float dy[N];
+                for (int p = 0; p < N; ++p) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(ys + p * TT * ROW + roff);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                    for (int p = 0; p < N; ++p) dy[p] = ld_bf16(ys + p * TT * ROW + roff);
+                    for (int e = 0; e < 4; ++e) { dyf[p][2 * e] = bf_lo(ww[e]); dyf[p][2 * e + 1] = bf_hi(ww[e]); }
+                }
 #pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const int i = 2 * b + ih;
-                        if (i < N) {
-                            const float4 ca = *reinterpret_cast<const float4*>(cs + sw128_off(tl, 2 * i));
-                            const float4 cb = *reinterpret_cast<const float4*>(cs + sw128_off(tl, 2 * i + 1));
-                            const float cr[4] = {ca.y, ca.z, ca.w, cb.x};
-                            const float xv = ld_bf16(xs + i * TT * ROW + roff);
-                            float v = fmaf(ca.x, dxv, __uint_as_float(pg[b][u]));
-                            v = fmaf(cb.y, xv, v);
+                for (int j = 0; j < 2; ++j) {
+                    const int i = 2 * hp + j;
+                    if (i >= N) continue;
+                    const uint4 w = *reinterpret_cast<const uint4*>(xs + i * TT * ROW + roff);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    float o[8];
 #pragma unroll
-                            for (int p = 0; p < N; ++p) v = fmaf(cr[p], dy[p], v);
-                            if (t < t_hi) dX[((int64_t)t * N + i) * d + c0 + c] = __float2bfloat16(v);
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        const float xv = (e & 1) ? bf_hi(ww[e >> 1]) : bf_lo(ww[e >> 1]);
+                        const uint32_t pv = j ? pg1[8 * cc + e] : pg0[8 * cc + e];
+                        float v = fmaf(cf[j][0], dxf[e], __uint_as_float(pv));
+                        v = fmaf(cf[j][5], xv, v);
+#pragma unroll
+                        for (int p = 0; p < N; ++p) v = fmaf(cf[j][1 + p], dyf[p][e], v);
+                        o[e] = v;
+                    }
+                    if (t < t_hi) {
+                        const uint4 out = make_uint4(pack_f32x2(o[0], o[1]), pack_f32x2(o[2], o[3]),
+                                                     pack_f32x2(o[4], o[5]), pack_f32x2(o[6], o[7]));
+                        *reinterpret_cast<uint4*>(dX + ((int64_t)t * N + i) * d + c0 + cb + 8 * cc) = out;
                     }
                 }
             }
@@ -333,17 +394,16 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi, 
                 mbar_arrive(bar(B_EMPTY + st));
             }
         }
-        // dphi partials of the group: warp half h reads block h (its last phi G wait covered
-        // every MMA of the CTA)
-        const int b = h;
-        if (ok && b < NB) {
-            const int i = 2 * b + ih;
+        // dphi partials of the group: warp half h reads block h (TMEM lane = row k of the block;
+        // the last phi G wait covered every MMA of the CTA)
+        if (ok && h < NB) {
+            const int i = 2 * h + (q >> 1), c = 32 * (q & 1) + lane;
             if (i < N) {
                 float* dst = part + ((int64_t)g * K + (int64_t)i * d + c0 + c) * M;
                 if (nst > 0) {
                     float vh[32], vl[32];
-                    tmem_ld32(tm + lane_base + C::DPHI_COL + 64 * b, vh);
-                    tmem_ld32(tm + lane_base + C::DPHI_COL + 64 * b + 32, vl);
+                    tmem_ld32(tq + C::DPHI_COL + 64 * h, vh);
+                    tmem_ld32(tq + C::DPHI_COL + 64 * h + 32, vl);
 #pragma unroll
                     for (int j = 0; j < M; ++j) dst[j] = vh[j] + vl[j];
                 } else {
@@ -416,19 +476,20 @@ cudaError_t launch_n(const BwdArgs& a, const void* rec, float* part, int groups,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
-    {   // records: dims (e, t, row), strides t: 384 B, row: 128 B
-        const cuuint64_t dims[3] = {64, (cuuint64_t)a.T, 3};
-        const cuuint64_t str[2] = {(cuuint64_t)BWD_REC_BYTES, 128};
-        const cuuint32_t box[3] = {64, TT, 3};
-        r = enc(&maps.rec, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(rec), dims, str, box, e1,
+    {   // G rows of the records: dims (e, t), stride t: one record
+        const cuuint64_t dims[2] = {64, (cuuint64_t)a.T};
+        const cuuint64_t str[1] = {(cuuint64_t)BWD_REC_BYTES};
+        const cuuint32_t box[2] = {64, TT};
+        r = enc(&maps.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(rec), dims, str, box, e1,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
     const int slices = a.d / CW;
     const unsigned grid = (unsigned)(slices * groups);
-    bwd_tc_kernel<N><<<grid, THREADS, Cfg<N>::SMEM, a.stream>>>(maps, a.phi, (int)a.T, a.d, (int)tpg,
-                                                                static_cast<__nv_bfloat16*>(a.dX), part);
+    bwd_tc_kernel<N><<<grid, THREADS, Cfg<N>::SMEM, a.stream>>>(
+        maps, a.phi, static_cast<const unsigned char*>(rec), (int)a.T, a.d, (int)tpg,
+        static_cast<__nv_bfloat16*>(a.dX), part);
     return cudaGetLastError();
 }
 

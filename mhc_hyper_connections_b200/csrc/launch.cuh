@@ -111,10 +111,10 @@ BwdLayout backward_layout(int64_t T, int n, int d, bool tc);
 int64_t backward_workspace_floats(int64_t T, int n, int d);
 
 // Tensor-core dX / dphi step (backward_tc.cu): bf16, n <= 4, d a multiple of 64.  It reads one
-// record of BWD_REC_BYTES per token, written by the token kernel: row 0 = [G_hi | G_lo], row 1
-// = [G_hi | 0] (bf16, 32 each, zero past m), row 2 = per stream i < 4 the fp32 coefficients
+// record of BWD_REC_BYTES per token, written by the token kernel: bytes 0-127 = [G_hi | G_lo]
+// (bf16, 32 each, zero past m), bytes 128-255 = per stream i < 4 the fp32 coefficients
 // {H_pre[i], H_res[0..3][i], -beta, 0, 0} (zero past n).
-constexpr int BWD_REC_BYTES = 384;
+constexpr int BWD_REC_BYTES = 256;
 constexpr int BWD_TC_SMS = 148;   // groups are sized for this many SMs (results do not depend on the device)
 bool bwd_tc_shape_ok(int64_t T, int n, int d, DType dt);
 bool bwd_tc_device_ok(int n);
