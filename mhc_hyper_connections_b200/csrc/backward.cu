@@ -137,7 +137,19 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
                  float* __restrict__ G, float* __restrict__ beta, unsigned char* __restrict__ rec) {
     constexpr int M = N * N + 2 * N, NR = red_len(N);
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= Tn) return;
+    if (t >= Tn) {
+        // the tensor-core step's records of the last tile's rows past T are zero
+        if (rec != nullptr && t < (Tn + BWD_REC_TILE - 1) / BWD_REC_TILE * BWD_REC_TILE) {
+            unsigned char* tile = rec + t / BWD_REC_TILE * (BWD_REC_TILE * BWD_REC_BYTES);
+            const int r = (int)(t % BWD_REC_TILE);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                *reinterpret_cast<uint4*>(tile + r * 128 + j * 16) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(tile + 8192 + r * 128 + j * 16) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        return;
+    }
     const float* Rt = R + t * NR;
     float hh[M], out[M];
 #pragma unroll
@@ -244,8 +256,13 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         beta[t] = bt;
         return;
     }
-    // the tensor-core step's record (launch.cuh): [G_hi | G_lo], then the coefficients
-    uint4* r4 = reinterpret_cast<uint4*>(rec + t * BWD_REC_BYTES);
+    // the tensor-core step's records (launch.cuh): row r of the token's tile, 16-byte chunk j
+    // at position j ^ (r % 8), G row in the first half of the tile, coefficients in the second
+    unsigned char* tile = rec + t / BWD_REC_TILE * (BWD_REC_TILE * BWD_REC_BYTES);
+    const int r = (int)(t % BWD_REC_TILE);
+    auto chunk = [&](int half, int j) {
+        return reinterpret_cast<uint4*>(tile + half * 8192 + r * 128 + ((j ^ (r & 7)) << 4));
+    };
     uint32_t w[32];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -261,8 +278,7 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
         w[16 + e] = (uint32_t)__bfloat16_as_ushort(lv[0]) | ((uint32_t)__bfloat16_as_ushort(lv[1]) << 16);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) r4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-    float4* c4 = reinterpret_cast<float4*>(rec + t * BWD_REC_BYTES + 128);
+    for (int j = 0; j < 8; ++j) *chunk(0, j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         float cf[8];
@@ -274,8 +290,10 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
             for (int p = 0; p < N; ++p) cf[1 + p] = H[t * M + N + p * N + i];
             cf[5] = -bt;
         }
-        c4[2 * i] = make_float4(cf[0], cf[1], cf[2], cf[3]);
-        c4[2 * i + 1] = make_float4(cf[4], cf[5], cf[6], cf[7]);
+        *chunk(1, 2 * i) = make_uint4(__float_as_uint(cf[0]), __float_as_uint(cf[1]), __float_as_uint(cf[2]),
+                                      __float_as_uint(cf[3]));
+        *chunk(1, 2 * i + 1) = make_uint4(__float_as_uint(cf[4]), __float_as_uint(cf[5]), __float_as_uint(cf[6]),
+                                          __float_as_uint(cf[7]));
     }
 }
 
@@ -444,7 +462,8 @@ cudaError_t launch_n(const BwdArgs& a, const BwdLayout& L) {
             X, static_cast<const T*>(a.F), dY, dxi, a.H, Tn, d, R, static_cast<T*>(a.dF_out));
     }
     unsigned char* rec = L.tc ? reinterpret_cast<unsigned char*>(ws + L.off_rec) : nullptr;
-    bwd_token_kernel<N><<<(unsigned)((Tn + TOK_THREADS - 1) / TOK_THREADS), TOK_THREADS, 0, a.stream>>>(
+    const int64_t tok_threads = L.tc ? (Tn + BWD_REC_TILE - 1) / BWD_REC_TILE * BWD_REC_TILE : Tn;
+    bwd_token_kernel<N><<<(unsigned)((tok_threads + TOK_THREADS - 1) / TOK_THREADS), TOK_THREADS, 0, a.stream>>>(
         R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res, Tn, K, a.eps, a.t_max, dl, G, beta, rec);
     if (L.tc) {
         e = launch_bwd_tc(a, rec, part, L.groups, L.tokens_per_group);
@@ -501,7 +520,7 @@ BwdLayout backward_layout(int64_t T, int n, int d, bool tc) {
     L.off_R = off;      off += up(T * red_len(n));
     L.off_dl = off;     off += up(T * m);
     if (L.tc) {
-        L.off_rec = off; off += up(T * (BWD_REC_BYTES / 4));
+        L.off_rec = off; off += up((T + BWD_REC_TILE - 1) / BWD_REC_TILE * BWD_REC_TILE * (BWD_REC_BYTES / 4));
     } else {
         L.off_G = off;      off += up(T * m);
         L.off_beta = off;   off += up(T);

@@ -110,11 +110,14 @@ BwdLayout backward_layout(int64_t T, int n, int d, bool tc);
 // workspace the backward needs whichever dX / dphi kernel it takes, in floats
 int64_t backward_workspace_floats(int64_t T, int n, int d);
 
-// Tensor-core dX / dphi step (backward_tc.cu): bf16, n <= 4, d a multiple of 64.  It reads one
-// record of BWD_REC_BYTES per token, written by the token kernel: bytes 0-127 = [G_hi | G_lo]
-// (bf16, 32 each, zero past m), bytes 128-255 = per stream i < 4 the fp32 coefficients
-// {H_pre[i], H_res[0..3][i], -beta, 0, 0} (zero past n).
+// Tensor-core dX / dphi step (backward_tc.cu): bf16, n <= 4, d a multiple of 64.  It reads, per
+// tile of BWD_REC_TILE tokens (token t in tile t / 64, row r = t % 64), a block of records written
+// by the token kernel: bytes [0, 8192) hold row r's [G_hi | G_lo] (bf16, 32 each, zero past m)
+// and bytes [8192, 16384) row r's per-stream fp32 coefficients {H_pre[i], H_res[0..3][i], -beta,
+// 0, 0} for i < 4 (zero past n); each 128-byte row stores its 16-byte chunk j at position
+// j ^ (r % 8), the 128-byte swizzle the MMA reads.  Rows past T are zero.
 constexpr int BWD_REC_BYTES = 256;
+constexpr int BWD_REC_TILE = 64;
 constexpr int BWD_TC_SMS = 148;   // groups are sized for this many SMs (results do not depend on the device)
 bool bwd_tc_shape_ok(int64_t T, int n, int d, DType dt);
 bool bwd_tc_device_ok(int n);
