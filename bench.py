@@ -43,12 +43,16 @@ FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
 # the named kernel on the headline workload, with the sha256 of the kernel source it was
 # measured on; reported as null once that source changes.
 NCU_TRAFFIC = {
-    # measured at T=8192 (X = 256 MiB, twice the L2) and scaled x2 to T=16384
-    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.162176 + 50.852096) * 2e6), "36fc8e56023222c5"),
-    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.358144 + 213.037056) * 2e6), "96dbcd70460419e6"),
-    # the six launches of one mhc_backward call, captured at T=16384 itself (on the file's
-    # previous hash 8883e6aea5058f0e: since then only its header comment changed)
-    ("backward", "bf16_T16384_n4_d4096_outliers"): (2595701760 + 615055104, "2fad304296d6ff37"),
+    # dram__bytes_read.sum + dram__bytes_write.sum per launch, captured at half the token count
+    # (X still twice the L2) and scaled x2 (profiles/ holds the commands and the raw counts)
+    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.129920 + 41.285632) * 2e6), "157c4df346643206"),
+    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.353792 + 209.392128) * 2e6), "96dbcd70460419e6"),
+    # the three launches of the two-pass path at T=4096: the projection and read-map kernels
+    # scaled x2, the phi packing (no token dependence) once
+    ("pre", "bf16_T8192_n8_d4096"): (int(((279.564032 + 0.481536 + 268.976384 + 5.803520) * 2 + 10.491392) * 1e6),
+                                     "c345c599d98f4053"),
+    # the six launches of one mhc_backward call at T=8192, scaled x2 (backward.cu + backward_tc.cu)
+    ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.777344 + 251.888640) * 2e6), "71c8ad0dd3057bf4"),
 }
 
 
@@ -63,11 +67,15 @@ def _hbm_peak():
 
 
 def _src_sha(rel):
+    """sha256 prefix of a source file, or of several (a list) read one after another."""
+    h = hashlib.sha256()
     try:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            return hashlib.sha256(f.read()).hexdigest()[:16]
+        for r in ([rel] if isinstance(rel, str) else rel):
+            with open(os.path.join(ROOT, r), "rb") as f:
+                h.update(f.read())
     except OSError:
         return None
+    return h.hexdigest()[:16]
 
 
 def bytes_per_token(n, d, es):
@@ -554,9 +562,10 @@ def run_backward(args, rank, world, local_rank):
     bw_gbs = by_bwd * T / (st[2] / 1e3) / 1e9
     step_bytes = (by_pre + by_post + by_bwd) * T
     step_gbs = step_bytes / (ms_total / 1e3 / K) / 1e9       # per GPU: each processes T tokens
-    bwd_src = "mhc_hyper_connections_b200/csrc/backward.cu"
+    bwd_srcs = ["mhc_hyper_connections_b200/csrc/backward.cu", "mhc_hyper_connections_b200/csrc/backward_tc.cu"]
+    bwd_src = " + ".join(bwd_srcs)
     rec = NCU_TRAFFIC.get(("backward", args.config))
-    traffic = rec[0] if (rec and not args.tokens and rec[1] == _src_sha(bwd_src)) else None
+    traffic = rec[0] if (rec and not args.tokens and rec[1] == _src_sha(bwd_srcs)) else None
     line = {
         "metric": "mHC forward+backward tokens/s (pre_train + post + backward), n=4 d=4096 bf16",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
