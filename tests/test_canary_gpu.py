@@ -63,7 +63,7 @@ def test_forward_writes_stay_inside_their_outputs(T, n, d, dt):
 
 
 @pytest.mark.parametrize("T,n,d,dt", [(100, 3, 136, "bf16"), (33, 2, 24, "f32"), (300, 1, 1024, "bf16"),
-                                      (700, 4, 512, "bf16")])
+                                      (700, 4, 512, "bf16"), (129, 3, 192, "bf16"), (65, 2, 64, "bf16")])
 def test_training_writes_stay_inside_their_outputs(T, n, d, dt):
     w = wl.make_inputs(T=T, n=n, d=d, dtype=dt, seed=2 * T + d, alpha=0.3)
     t = torch_inputs(w, device=DEV)
