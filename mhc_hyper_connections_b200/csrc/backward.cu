@@ -390,45 +390,62 @@ bwd_dphi_sum_kernel(const float* __restrict__ part, int64_t len, int groups, flo
     }
 }
 
-// Column j (one CTA each): colsum[j] = sum_t dl[t][j] and colsum[M + j] = sum_t dl[t][j] h[t][j];
-// each thread sums a fixed strided set of tokens, then a fixed-order tree.
+// Column sums over the tokens, in two fixed-order levels.  Partition p (one CTA) covers tokens
+// [p * per, (p + 1) * per): thread (u, j), u < CS_ROWS, adds dl[t][j] and dl[t][j] h[t][j] over
+// t = start + u, start + u + CS_ROWS, ... (consecutive threads read consecutive floats of a
+// row), then the CS_ROWS lanes of a column are added in order into part[p][j], part[p][M + j].
+constexpr int CS_PARTS = 64;
+template <int M>
 __global__ void __launch_bounds__(SUM_THREADS)
-bwd_colsum_kernel(const float* __restrict__ dl, const float* __restrict__ h, int64_t Tn, int M,
-                  float* __restrict__ colsum) {
-    __shared__ float s0[SUM_THREADS], s1[SUM_THREADS];
-    const int j = blockIdx.x;
-    float a = 0.f, b = 0.f;
-    for (int64_t t = threadIdx.x; t < Tn; t += SUM_THREADS) {
-        const float v = dl[t * M + j];
-        a += v;
-        b = fmaf(v, h[t * M + j], b);
-    }
-    s0[threadIdx.x] = a;
-    s1[threadIdx.x] = b;
-    __syncthreads();
-    for (int w = SUM_THREADS / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) {
-            s0[threadIdx.x] += s0[threadIdx.x + w];
-            s1[threadIdx.x] += s1[threadIdx.x + w];
+bwd_colsum_part_kernel(const float* __restrict__ dl, const float* __restrict__ h, int64_t Tn, int64_t per,
+                       float* __restrict__ part) {
+    constexpr int CS_ROWS = SUM_THREADS / M;
+    __shared__ float s0[CS_ROWS][M], s1[CS_ROWS][M];
+    const int u = threadIdx.x / M, j = threadIdx.x % M;
+    const int64_t t0 = (int64_t)blockIdx.x * per;
+    const int64_t t1 = t0 + per < Tn ? t0 + per : Tn;
+    if (u < CS_ROWS) {
+        float a = 0.f, b = 0.f;
+        for (int64_t t = t0 + u; t < t1; t += CS_ROWS) {
+            const float v = dl[t * M + j];
+            a += v;
+            b = fmaf(v, h[t * M + j], b);
         }
-        __syncthreads();
+        s0[u][j] = a;
+        s1[u][j] = b;
     }
-    if (threadIdx.x == 0) {
-        colsum[j] = s0[0];
-        colsum[M + j] = s1[0];
+    __syncthreads();
+    if (threadIdx.x < M) {
+        float a = 0.f, b = 0.f;
+#pragma unroll 1
+        for (int r = 0; r < CS_ROWS; ++r) {
+            a += s0[r][threadIdx.x];
+            b += s1[r][threadIdx.x];
+        }
+        part[(int64_t)blockIdx.x * 2 * M + threadIdx.x] = a;
+        part[(int64_t)blockIdx.x * 2 * M + M + threadIdx.x] = b;
     }
 }
 
-// db from the column sums; dalpha = (pre, post, res) sums of the dl * h column sums.
-__global__ void bwd_bias_alpha_kernel(const float* __restrict__ colsum, int n, float* __restrict__ db_pre,
-                                      float* __restrict__ db_post, float* __restrict__ db_res,
-                                      float* __restrict__ dalpha) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    const int nn = n * n, M = nn + 2 * n;
+// The partitions' sums added in partition order; db from the dl sums, dalpha = (pre, post, res)
+// sums of the dl * h sums.
+template <int N>
+__global__ void bwd_colsum_final_kernel(const float* __restrict__ part, int parts, float* __restrict__ db_pre,
+                                        float* __restrict__ db_post, float* __restrict__ db_res,
+                                        float* __restrict__ dalpha) {
+    constexpr int M = N * N + 2 * N;
+    __shared__ float cs[2 * M];
+    for (int q = threadIdx.x; q < 2 * M; q += blockDim.x) {
+        float a = 0.f;
+        for (int p = 0; p < parts; ++p) a += part[(int64_t)p * 2 * M + q];
+        cs[q] = a;
+    }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
     float ap = 0.f, ar = 0.f, aq = 0.f;
-    for (int j = 0; j < n; ++j) { db_pre[j] = colsum[j]; ap += colsum[M + j]; }
-    for (int q = 0; q < nn; ++q) { db_res[q] = colsum[n + q]; ar += colsum[M + n + q]; }
-    for (int j = 0; j < n; ++j) { db_post[j] = colsum[n + nn + j]; aq += colsum[M + n + nn + j]; }
+    for (int j = 0; j < N; ++j) { db_pre[j] = cs[j]; ap += cs[M + j]; }
+    for (int q = 0; q < N * N; ++q) { db_res[q] = cs[N + q]; ar += cs[M + N + q]; }
+    for (int j = 0; j < N; ++j) { db_post[j] = cs[N + N * N + j]; aq += cs[M + N + N * N + j]; }
     dalpha[0] = ap;
     dalpha[1] = aq;
     dalpha[2] = ar;
@@ -480,8 +497,12 @@ cudaError_t launch_n(const BwdArgs& a, const BwdLayout& L) {
         if (blocks > (int64_t)di.sm_count * 8) blocks = (int64_t)di.sm_count * 8;
         bwd_dphi_sum_kernel<<<(unsigned)blocks, SUM_THREADS, 0, a.stream>>>(part, len, L.groups, a.dphi);
     }
-    bwd_colsum_kernel<<<M, SUM_THREADS, 0, a.stream>>>(dl, a.h, Tn, M, colsum);
-    bwd_bias_alpha_kernel<<<1, 32, 0, a.stream>>>(colsum, N, a.db_pre, a.db_post, a.db_res, a.dalpha);
+    {
+        const int64_t per = (Tn + CS_PARTS - 1) / CS_PARTS;
+        bwd_colsum_part_kernel<M><<<CS_PARTS, SUM_THREADS, 0, a.stream>>>(dl, a.h, Tn, per, colsum);
+        bwd_colsum_final_kernel<N><<<1, 64, 0, a.stream>>>(colsum, CS_PARTS, a.db_pre, a.db_post, a.db_res,
+                                                           a.dalpha);
+    }
     return cudaGetLastError();
 }
 
@@ -526,7 +547,7 @@ BwdLayout backward_layout(int64_t T, int n, int d, bool tc) {
         L.off_beta = off;   off += up(T);
     }
     L.off_part = off;   off += up((int64_t)L.groups * K * m);
-    L.off_colsum = off; off += up(2 * m);
+    L.off_colsum = off; off += up(CS_PARTS * 2 * m);   // the column sums' partitions
     L.floats = off;
     return L;
 }
