@@ -55,6 +55,7 @@ constexpr int SW = 2;              // atoms per stage (one 64 KB box of X, one c
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
 static_assert(TPO % 32 == 0, "the owner warp takes TPO / 32 tokens per lane");
+static_assert(THREADS == 4 * TPO && TPO % NWARPS == 0, "the last tile's maps: four threads per owned token");
 
 template <int N>
 struct Cfg {
@@ -64,6 +65,8 @@ struct Cfg {
     static constexpr int PHI_ATOM = NB / 8 * 1024;         // bytes of one packed atom
     static constexpr int W = ((MH > M + 1 ? MH : M + 1) + 3) / 4 * 4;   // floats per partial record
     static constexpr int STAGE = SW * (X_STAGE + PHI_ATOM);
+    static constexpr int HSW = W | 1;                      // owner buffer row stride (odd: no bank conflicts)
+    static constexpr int HS = 32 * HSW * 4;                // owner: summed records of 32 tokens
     static constexpr int NACCB = TMEM_COLS / (2 * NB) >= 2 ? 2 : 1;     // accumulator buffers
     static_assert(NB <= 256 && NB % 16 == 0, "MMA N for M = 128");
     static_assert(2 * NB <= TMEM_COLS, "both halves fit TMEM");
@@ -157,6 +160,101 @@ wide_pack_kernel(const float* __restrict__ phi, int ka_total, uint8_t* __restric
 }
 
 // ---------------------------------------------------------------- 2. projection
+// The maps of one token from its summed projection hv (length m, not yet divided by r), four
+// lanes per token ("DeepSeek-V4/mhc", equations a/b/c-tilde, gate, sinkhorn-init, sinkhorn;
+// the HC maps b + alpha tanh(h / r) when hc): lane gl of the group owns rows 2 gl and 2 gl + 1
+// (those below N).  In each Sinkhorn round a column sum adds the lanes' two-row sums by xor
+// shuffles within the group (every lane gets the same sum); row sums are the lane's own.  All
+// four lanes run the shuffles; only `valid` tokens are written.
+template <int N>
+__device__ __forceinline__ void owner_maps4(const float* hv, float inv_r, int gl, const float* b_pre,
+                                            const float* b_post, const float* b_res, float a_pre, float a_post,
+                                            float a_res, int t_max, bool hc, bool valid, float* Hrow, float* hrow) {
+    static_assert(N <= 8, "two rows per lane, four lanes per token");
+    float Mx[2][N];
+    bool own[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int i = 2 * gl + r;
+        own[r] = i < N;
+#pragma unroll
+        for (int j = 0; j < N; ++j)
+            Mx[r][j] = (own[r] && !hc) ? expf(a_res * (hv[N + i * N + j] * inv_r) + b_res[i * N + j]) : 0.f;
+    }
+    if (!hc) {
+        for (int it = 0; it < t_max; ++it) {
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                float s = Mx[0][j] + Mx[1][j];
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                const float inv = 1.0f / s;
+                Mx[0][j] *= inv;
+                Mx[1][j] *= inv;
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (!own[r]) continue;
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < N; ++j) s += Mx[r][j];
+                const float inv = 1.0f / s;
+#pragma unroll
+                for (int j = 0; j < N; ++j) Mx[r][j] *= inv;
+            }
+        }
+    }
+    if (!valid) return;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (!own[r]) continue;
+        const int i = 2 * gl + r;
+        const float zp = hv[i] * inv_r, zq = hv[N + N * N + i] * inv_r;
+        Hrow[i] = hc ? b_pre[i] + a_pre * tanhf(zp) : sigmoid_f32(a_pre * zp + b_pre[i]);
+        Hrow[N + N * N + i] = hc ? b_post[i] + a_post * tanhf(zq) : 2.0f * sigmoid_f32(a_post * zq + b_post[i]);
+#pragma unroll
+        for (int j = 0; j < N; ++j)
+            Hrow[N + i * N + j] = hc ? b_res[i * N + j] + a_res * tanhf(hv[N + i * N + j] * inv_r) : Mx[r][j];
+        if (hrow != nullptr) {
+            hrow[i] = zp;
+            hrow[N + N * N + i] = zq;
+#pragma unroll
+            for (int j = 0; j < N; ++j) hrow[N + i * N + j] = hv[N + i * N + j] * inv_r;
+        }
+    }
+}
+
+// The C partial records of tokens [u0, u0 + nu) of a tile added in source order, the lanes along
+// the record (coalesced loads), into rows u0.. of hs (row stride HSW).
+template <int W, int HSW>
+__device__ __forceinline__ void sum_records(const float* __restrict__ blk, int rank, int u0, int nu, int lane,
+                                            float* hs, int hs_row0) {
+    constexpr int QW = (W + 31) / 32;
+#pragma unroll 1
+    for (int v0 = 0; v0 < nu; v0 += 4) {
+        float acc[4][QW];
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+            const float* rec = blk + ((int64_t)(rank * TPO + u0 + v0 + uu) * C) * W;
+#pragma unroll
+            for (int q = 0; q < QW; ++q) {
+                const int j = lane + 32 * q;
+                float v = 0.f;
+                if (j < W && v0 + uu < nu) {
+#pragma unroll
+                    for (int src = 0; src < C; ++src) v += __ldcg(rec + src * W + j);
+                }
+                acc[uu][q] = v;
+            }
+        }
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu)
+#pragma unroll
+            for (int q = 0; q < QW; ++q)
+                if (lane + 32 * q < W && v0 + uu < nu) hs[(hs_row0 + v0 + uu) * HSW + lane + 32 * q] = acc[uu][q];
+    }
+}
+
 template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
 wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__ packed,
@@ -167,7 +265,7 @@ wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__
                  int hc, unsigned long long wait_ns)
 {
     using Cf = Cfg<N>;
-    constexpr int M = Cf::M, MH = Cf::MH, NB = Cf::NB, W = Cf::W, NACCB = Cf::NACCB;
+    constexpr int M = Cf::M, MH = Cf::MH, NB = Cf::NB, W = Cf::W, NACCB = Cf::NACCB, HSW = Cf::HSW;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -181,6 +279,7 @@ wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__
     const uint32_t o_misc = o_bar + B_COUNT * 8u;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sb + o_misc);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sb + o_misc + 4);
+    float* hs = reinterpret_cast<float*>(sb + o_misc + 16);
     auto bar = [&](int i) -> uint32_t { return base + o_bar + 8u * (uint32_t)i; };
     const Waiter wait{abort_flag, wait_ns};
     const Waiter drain{abort_flag, wait_ns > kWaitNs ? wait_ns : kWaitNs};
@@ -365,47 +464,65 @@ wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__
             }
         }
     } else if (warp == 3) {
-        // owner: tokens rank * TPO + lane + 32 j of every tile; adds the C partial records of
-        // a token in source order
-        for (int k = 0; k < my_tiles; ++k) {
+        // owner of every tile but the last (whose owner phase all warps share, below): tokens
+        // rank * TPO .. rank * TPO + TPO - 1, 32 at a time, record sums into hs, then the maps
+        // one lane per token
+        for (int k = 0; k + 1 < my_tiles; ++k) {
             const int sl = k % NS, us = k / NS;
             if (!wait.template operator()<true>(bar(B_PFULL + sl), us & 1, E_PFULL)) break;
             const int tile = cid + k * ncl;
+            const float* blk = scratch + (int64_t)tile * TT * C * W;
 #pragma unroll 1
-            for (int j32 = 0; j32 < TPO / 32; ++j32) {
-                const int t = (int)rank * TPO + j32 * 32 + lane;
-                const float* rec = scratch + ((int64_t)tile * TT + t) * C * W;
-                float hv[M];
-                float ssum = 0.f;
-#pragma unroll
-                for (int j = 0; j < M; ++j) hv[j] = 0.f;
-#pragma unroll 1
-                for (int src = 0; src < C; ++src) {
-                    const float* r = rec + src * W;
-#pragma unroll
-                    for (int j = 0; j < M; ++j) hv[j] += __ldcg(r + j);
-                    ssum += __ldcg(r + M);
-                }
-                if (j32 == TPO / 32 - 1) {   // every record of this tile has been read
+            for (int half = 0; half < TPO / 32; ++half) {
+                sum_records<W, HSW>(blk, (int)rank, half * 32, 32, lane, hs, 0);
+                if (half == TPO / 32 - 1) {   // every record of this tile has been read
                     __syncwarp();
                     if (lane < C) mbar_arrive_remote(mapa(bar(B_PEMPTY + sl), (uint32_t)lane));
                 }
-                const int64_t tok = (int64_t)tile * TT + t;
-                const float inv_r = 1.0f / sqrtf(ssum / (float)(N * d) + eps);
-#pragma unroll
-                for (int j = 0; j < M; ++j) hv[j] *= inv_r;
+                __syncwarp();                 // hs is complete before the maps read it
+                const int64_t tok = (int64_t)tile * TT + (int)rank * TPO + half * 32 + lane;
+                const float* hv = hs + lane * HSW;
+                const float inv_r = 1.0f / sqrtf(hv[M] / (float)(N * d) + eps);
                 if (tok < T) {
                     if (h_out != nullptr) {
 #pragma unroll
-                        for (int j = 0; j < M; ++j) h_out[tok * M + j] = hv[j];
+                        for (int j = 0; j < M; ++j) h_out[tok * M + j] = hv[j] * inv_r;
                     }
                     float out[M];
-                    if (hc) token_maps_hc<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, out);
-                    else token_maps<N>(hv, 1.0f, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
+                    if (hc) token_maps_hc<N>(hv, inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, out);
+                    else token_maps<N>(hv, inv_r, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, out);
 #pragma unroll
                     for (int j = 0; j < M; ++j) H[tok * M + j] = out[j];
                 }
+                __syncwarp();                 // the maps have read hs before the next half fills it
             }
+        }
+    }
+
+    // ---- the last tile's owner phase, all warps: the stage ring is idle once every role has
+    // left its loop (loads drained, MMAs complete), so it holds the 64 tokens' summed records;
+    // each warp sums 8 tokens' records, then four threads form each token's maps
+    if (my_tiles > 0) {
+        const int k = my_tiles - 1, sl = k % NS, us = k / NS;
+        volatile int* go = reinterpret_cast<volatile int*>(sb + o_misc + 8);
+        if (warp == 3) {
+            const bool ok = !*abort_flag && wait.template operator()<true>(bar(B_PFULL + sl), us & 1, E_PFULL);
+            if (lane == 0) *go = ok ? 1 : 0;
+        }
+        __syncthreads();
+        if (*go) {
+            const int tile = cid + k * ncl;
+            float* hsl = reinterpret_cast<float*>(sb);
+            sum_records<W, HSW>(scratch + (int64_t)tile * TT * C * W, (int)rank, warp * (TPO / NWARPS),
+                                TPO / NWARPS, lane, hsl, warp * (TPO / NWARPS));
+            __syncthreads();
+            if (warp == 3 && lane < C) mbar_arrive_remote(mapa(bar(B_PEMPTY + sl), (uint32_t)lane));
+            const int u = threadIdx.x >> 2, gl = threadIdx.x & 3;
+            const int64_t tok = (int64_t)tile * TT + (int)rank * TPO + u;
+            const float* hv = hsl + u * HSW;
+            const float inv_r = 1.0f / sqrtf(hv[M] / (float)(N * d) + eps);
+            owner_maps4<N>(hv, inv_r, gl, b_pre, b_post, b_res, a_pre, a_post, a_res, t_max, hc != 0, tok < T,
+                           H + tok * M, h_out != nullptr ? h_out + tok * M : nullptr);
         }
     }
 
@@ -463,7 +580,7 @@ struct Plan {
 };
 
 template <int N>
-int smem_bytes(int nstage) { return nstage * Cfg<N>::STAGE + B_COUNT * 8 + 16 + 1024; }
+int smem_bytes(int nstage) { return nstage * Cfg<N>::STAGE + B_COUNT * 8 + 16 + Cfg<N>::HS + 1024; }
 
 template <int N>
 Plan make_plan() {
