@@ -182,26 +182,35 @@ __device__ __forceinline__ void owner_maps4(const float* hv, float inv_r, int gl
             Mx[r][j] = (own[r] && !hc) ? expf(a_res * (hv[N + i * N + j] * inv_r) + b_res[i * N + j]) : 0.f;
     }
     if (!hc) {
+        // each step over all N columns at once, so the shuffles and divisions of different
+        // columns overlap
         for (int it = 0; it < t_max; ++it) {
+            float cs[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) cs[j] = Mx[0][j] + Mx[1][j];
+#pragma unroll
+            for (int j = 0; j < N; ++j) cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 1);
+#pragma unroll
+            for (int j = 0; j < N; ++j) cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 2);
+#pragma unroll
+            for (int j = 0; j < N; ++j) cs[j] = 1.0f / cs[j];
 #pragma unroll
             for (int j = 0; j < N; ++j) {
-                float s = Mx[0][j] + Mx[1][j];
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                const float inv = 1.0f / s;
-                Mx[0][j] *= inv;
-                Mx[1][j] *= inv;
+                Mx[0][j] *= cs[j];
+                Mx[1][j] *= cs[j];
             }
+            float rs[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                if (!own[r]) continue;
                 float s = 0.f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) s += Mx[r][j];
-                const float inv = 1.0f / s;
-#pragma unroll
-                for (int j = 0; j < N; ++j) Mx[r][j] *= inv;
+                rs[r] = own[r] ? 1.0f / s : 0.f;
             }
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int j = 0; j < N; ++j) Mx[r][j] *= rs[r];
         }
     }
     if (!valid) return;
