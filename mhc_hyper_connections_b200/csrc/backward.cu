@@ -105,7 +105,8 @@ bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __r
 
 // ---------------------------------------------------------------- K2
 // Column then row normalisation of A (one Sinkhorn round); cs, rs receive the reciprocals
-// of the column and row sums.
+// of the column and row sums (fast reciprocals, within 2 ulp: this replay only feeds the
+// gradient, whose tolerance is far wider).
 template <int N>
 __device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], float (&C)[N][N],
                                          float (&cs)[N], float (&rs)[N]) {
@@ -114,7 +115,7 @@ __device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], flo
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < N; ++i) s += A[i][j];
-        cs[j] = 1.0f / s;
+        cs[j] = __fdividef(1.0f, s);
 #pragma unroll
         for (int i = 0; i < N; ++i) B[i][j] = A[i][j] * cs[j];
     }
@@ -123,7 +124,7 @@ __device__ __forceinline__ void sk_round(float (&A)[N][N], float (&B)[N][N], flo
         float s = 0.f;
 #pragma unroll
         for (int j = 0; j < N; ++j) s += B[i][j];
-        rs[i] = 1.0f / s;
+        rs[i] = __fdividef(1.0f, s);
 #pragma unroll
         for (int j = 0; j < N; ++j) C[i][j] = B[i][j] * rs[i];
     }
