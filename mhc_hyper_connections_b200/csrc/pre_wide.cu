@@ -13,13 +13,15 @@
 //      the x_in buffer, which holds nothing else until launch 3 writes x_in.
 //   2. projection: clusters of C = 4 CTAs split K = n d; a cluster takes 256-token tiles
 //      (4-CTA clusters fill the GPU in one wave of tiles at the n = 8 workload).
-//      A stage holds two 64-channel atoms: the tile's X (one 64 KB TMA box) and those atoms
-//      of packed phi (one bulk copy, served from L2) -- large boxes, since one SM's TMA
-//      unit retires only a few boxes per microsecond.  Two warps issue tcgen05.mma
-//      (M = 128 tokens, N = 2 MH, K = 16), one per half of the tile, into TMEM; four warps
-//      add the tokens' squares.  Each CTA writes its partial projection and sum of squares
-//      of every token to a scratch block in the x_in buffer; the owner CTA of a token
-//      (64 tokens each) adds the 4 partials in a fixed order, applies 1/r and forms H.
+//      A stage holds one 64-channel atom: the tile's X (a 32 KB TMA box) and that atom of
+//      packed phi (a bulk copy, served from L2); four stages keep about 200 KB in flight per
+//      SM.  Two warps issue tcgen05.mma (M = 128 tokens, N = 2 MH, K = 16), one per half of
+//      the tile, into TMEM; four warps add the tokens' squares.  Each CTA writes its partial
+//      projection and sum of squares of every token to a scratch block in the x_in buffer;
+//      the owner CTA of a token (64 tokens each) adds the 4 partials in a fixed order into
+//      shared memory with coalesced loads, applies 1/r and forms H.  For a CTA's last tile
+//      every warp takes part (the stage ring is idle by then): four threads per token, the
+//      Sinkhorn rows split between them.
 //   3. read map: x_in = sum_i H_pre[i] X[i, :], streaming X from HBM a second time.
 //
 // X crosses HBM twice here; streaming phi instead against tiles small enough to re-read
@@ -51,7 +53,8 @@ constexpr int NWARPS = 8;          // 0 TMA, 1-2 MMA, 3 owner, 4-7 squares + epi
 constexpr int THREADS = NWARPS * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int X_STAGE = TT * 128;  // one atom of a 256-token tile
-constexpr int SW = 2;              // atoms per stage (one 64 KB box of X, one copy of phi)
+constexpr int SW = 1;              // atoms per stage (one 32 KB box of X, one copy of phi; measured
+                                   // slightly faster than two atoms per stage)
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
 static_assert(TPO % 32 == 0, "the owner warp takes TPO / 32 tokens per lane");
