@@ -300,6 +300,19 @@ mhc_status mhc_device_status(uint32_t* code);
  */
 mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us);
 
+/*
+ * mhc_debug_backward_stop_after -- test hook for the failure path of mhc_backward's
+ * tensor-core dX / dphi step (bf16, d a multiple of 64).  After this call its launches stop
+ * loading after `stages` 64-token stages per CTA (stages < 0: never, the default) and give
+ * up a wait after `wait_limit_us` microseconds (default 1000000; accepted range 1000 ..
+ * 10000000, else MHC_ERR_SHAPE).  Every stage before the stop completes (its dX tile is
+ * stored); the waits for the stage never loaded run into their limit, the step sets bits
+ * 24-31 in mhc_device_status, lets its copies and MMAs in flight complete and returns with dX
+ * and the parameter gradients incomplete.  Process-wide, from the next launch.  No
+ * counterpart on the pages: a library test facility for the bounded waits.
+ */
+mhc_status mhc_debug_backward_stop_after(int32_t stages, uint32_t wait_limit_us);
+
 /* Static English text for a status code (never NULL). */
 const char* mhc_status_string(mhc_status status);
 

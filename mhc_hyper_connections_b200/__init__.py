@@ -30,7 +30,7 @@ import threading
 __all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_post", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "mhc_amax_gain", "mhc_pre_path_for", "mhc_pre_path_ok", "mhc_device_status",
-           "mhc_debug_pre_stop_after",
+           "mhc_debug_pre_stop_after", "mhc_debug_backward_stop_after",
            "MhcError",
            "MHC_F32", "MHC_BF16", "PRE_AUTO", "PRE_GENERIC", "PRE_CLUSTER_TC", "PRE_TWO_PASS_TC", "library_path",
            "load_library", "EXPORTED_SYMBOLS"]
@@ -50,7 +50,8 @@ EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train
                     "mhc_pre_path_ok", "mhc_post",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
                     "mhc_amax_gain", "mhc_status_string",
-                    "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after")
+                    "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after",
+                    "mhc_debug_backward_stop_after")
 
 _lock = threading.Lock()
 _lib = None
@@ -111,6 +112,8 @@ def load_library():
         lib.mhc_device_status.restype = ci
         lib.mhc_debug_pre_stop_after.argtypes = [ctypes.c_int32, ctypes.c_uint32]
         lib.mhc_debug_pre_stop_after.restype = ci
+        lib.mhc_debug_backward_stop_after.argtypes = [ctypes.c_int32, ctypes.c_uint32]
+        lib.mhc_debug_backward_stop_after.restype = ci
         _lib = lib
     return _lib
 
@@ -390,6 +393,14 @@ def mhc_debug_pre_stop_after(tiles: int, wait_limit_us: int = 1_000_000) -> None
     loaded expire, the kernel returns early and mhc_device_status() reports it."""
     _check(load_library().mhc_debug_pre_stop_after(int(tiles), int(wait_limit_us)),
            "mhc_debug_pre_stop_after")
+
+
+def mhc_debug_backward_stop_after(stages: int, wait_limit_us: int = 1_000_000) -> None:
+    """Test hook of the backward's tensor-core dX / dphi step: later launches stop loading
+    after `stages` 64-token stages per CTA (stages < 0 restores normal operation) and give up
+    a wait after `wait_limit_us` microseconds; mhc_device_status() then reports bits 24-31."""
+    _check(load_library().mhc_debug_backward_stop_after(int(stages), int(wait_limit_us)),
+           "mhc_debug_backward_stop_after")
 
 
 def mhc_pre_path_ok(T: int, n: int, d: int, dtype, path: int) -> bool:

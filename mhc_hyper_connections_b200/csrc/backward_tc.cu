@@ -41,6 +41,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -214,7 +215,7 @@ template <int N>
 __global__ void __launch_bounds__(THREADS, 1)
 bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi,
               const unsigned char* __restrict__ rec, int T, int d, int tpg, __nv_bfloat16* __restrict__ dX,
-              float* __restrict__ part) {
+              float* __restrict__ part, int stop_stage, unsigned long long wait_ns) {
     using C = Cfg<N>;
     constexpr int M = C::M, NB = C::NB, NS = C::NS;
     extern __shared__ unsigned char smem_raw[];
@@ -224,8 +225,8 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi,
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
-    const Waiter wait{&abort_flag, kWaitNs};
-    const Waiter drain{&abort_flag, kDrainNs};
+    const Waiter wait{&abort_flag, wait_ns};
+    const Waiter drain{&abort_flag, wait_ns > kDrainNs ? wait_ns : kDrainNs};   // drains keep their full limit
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slices = d / CW;
@@ -302,6 +303,7 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi,
             int issued = 0, finished = 0;
             bool ok = true;
             for (int it = 0; it < nst; ++it) {
+                if (stop_stage >= 0 && it >= stop_stage) break;   // failure-path test hook
                 if (it >= NS) {
                     if (!(ok = finish(it - NS))) break;
                     finished = it - NS + 1;
@@ -510,6 +512,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// failure-path test hook (mhc_debug_backward_stop_after): stages per CTA after which the
+// producer stops loading (< 0: never), and the wait limit
+std::atomic<int> g_stop_stage{-1};
+std::atomic<unsigned long long> g_wait_ns{kWaitNs};
+
 template <int N>
 bool configure() {
     static int ok = -1;
@@ -563,7 +570,7 @@ cudaError_t launch_n(const BwdArgs& a, const void* rec, float* part, int groups,
     const unsigned grid = (unsigned)(slices * groups);
     bwd_tc_kernel<N><<<grid, THREADS, Cfg<N>::SMEM, a.stream>>>(
         maps, a.phi, static_cast<const unsigned char*>(rec), (int)a.T, a.d, (int)tpg,
-        static_cast<__nv_bfloat16*>(a.dX), part);
+        static_cast<__nv_bfloat16*>(a.dX), part, g_stop_stage.load(), g_wait_ns.load());
     return cudaGetLastError();
 }
 
@@ -605,6 +612,11 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, const void* rec, float* part, int gr
         case 4: return bwdtc::launch_n<4>(a, rec, part, groups, tpg);
         default: return cudaErrorInvalidValue;
     }
+}
+
+void bwd_tc_set_stop(int stop_stage, unsigned long long wait_ns) {
+    bwdtc::g_stop_stage.store(stop_stage);
+    bwdtc::g_wait_ns.store(wait_ns);
 }
 
 cudaError_t bwd_tc_status(unsigned* out, bool clear) {

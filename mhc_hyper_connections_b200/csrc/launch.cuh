@@ -125,6 +125,9 @@ int bwd_tc_groups(int64_t T, int d, int sm_count);
 int64_t bwd_tc_tokens_per_group(int64_t T, int groups);
 cudaError_t launch_bwd_tc(const BwdArgs& a, const void* rec, float* part, int groups, int64_t tpg);
 cudaError_t bwd_tc_status(unsigned* out, bool clear);
+// Failure-path test hook: launches after this call stop loading after `stop_stage` stages
+// per CTA (< 0: never) and give up a wait after `wait_ns`.
+void bwd_tc_set_stop(int stop_stage, unsigned long long wait_ns);
 
 // Amax Gain Magnitude of composite residual maps (diagnostics.cu).
 cudaError_t launch_amax_gain(const float* Hs, int L, int64_t T, int n, float* gain, cudaStream_t s);

@@ -346,6 +346,12 @@ mhc_status mhc_debug_pre_stop_after(int32_t tiles, uint32_t wait_limit_us) {
     return MHC_OK;
 }
 
+mhc_status mhc_debug_backward_stop_after(int32_t stages, uint32_t wait_limit_us) {
+    if (wait_limit_us < 1000u || wait_limit_us > 10000000u) return MHC_ERR_SHAPE;
+    bwd_tc_set_stop(stages < 0 ? -1 : (int)stages, (unsigned long long)wait_limit_us * 1000ull);
+    return MHC_OK;
+}
+
 mhc_status mhc_device_status(uint32_t* code) {
     if (!code) return MHC_ERR_NULL;
     unsigned v = 0, w = 0, b = 0;

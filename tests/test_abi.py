@@ -152,3 +152,6 @@ def test_debug_stop_hook_validation(lib):
     assert lib.mhc_debug_pre_stop_after(-1, 999) == 2
     assert lib.mhc_debug_pre_stop_after(3, 10_000_001) == 2
     assert lib.mhc_debug_pre_stop_after(-1, 1_000_000) == 0
+    assert lib.mhc_debug_backward_stop_after(-1, 999) == 2
+    assert lib.mhc_debug_backward_stop_after(3, 10_000_001) == 2
+    assert lib.mhc_debug_backward_stop_after(-1, 1_000_000) == 0
