@@ -50,6 +50,7 @@ bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __r
                   float* __restrict__ R, T* __restrict__ dF) {
     constexpr int M = N * N + 2 * N, NR = red_len(N), V = Vec16<T>::VEC;
     const int lane = threadIdx.x & 31;
+    pdl_wait();
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int nchunk = d / V;
     for (int64_t t = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < Tn; t += nwarps) {
@@ -138,6 +139,8 @@ bwd_token_kernel(const float* __restrict__ R, const float* __restrict__ H, const
                  float* __restrict__ G, float* __restrict__ beta, unsigned char* __restrict__ rec) {
     constexpr int M = N * N + 2 * N, NR = red_len(N);
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    pdl_launch_next();          // the dX / dphi step may set itself up meanwhile
+    pdl_wait();
     if (t >= Tn) {
         // the tensor-core step's records of the last tile's rows past T are zero
         if (rec != nullptr && t < (Tn + BWD_REC_TILE - 1) / BWD_REC_TILE * BWD_REC_TILE) {
@@ -324,6 +327,7 @@ bwd_dx_dphi_kernel(const T* __restrict__ X, const T* __restrict__ dY, const T* _
     }
     const int64_t t_lo = (int64_t)blockIdx.y * tpg;
     const int64_t t_hi = t_lo + tpg < Tn ? t_lo + tpg : Tn;
+    pdl_wait();
     for (int64_t tb = t_lo; tb < t_hi; tb += TB) {
         const int nb = (int)(t_hi - tb < TB ? t_hi - tb : TB);
         __syncthreads();
@@ -383,6 +387,7 @@ bwd_dx_dphi_kernel(const T* __restrict__ X, const T* __restrict__ dY, const T* _
 // dphi = sum over the token groups of the partials, in group order.
 __global__ void __launch_bounds__(SUM_THREADS)
 bwd_dphi_sum_kernel(const float* __restrict__ part, int64_t len, int groups, float* __restrict__ dphi) {
+    pdl_wait();
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < len;
          e += (int64_t)gridDim.x * blockDim.x) {
         float s = 0.f;
@@ -404,6 +409,7 @@ bwd_colsum_part_kernel(const float* __restrict__ dl, const float* __restrict__ h
     __shared__ float s0[CS_ROWS][M], s1[CS_ROWS][M];
     const int u = threadIdx.x / M, j = threadIdx.x % M;
     const int64_t t0 = (int64_t)blockIdx.x * per;
+    pdl_wait();
     const int64_t t1 = t0 + per < Tn ? t0 + per : Tn;
     if (u < CS_ROWS) {
         float a = 0.f, b = 0.f;
@@ -436,6 +442,7 @@ __global__ void bwd_colsum_final_kernel(const float* __restrict__ part, int part
                                         float* __restrict__ dalpha) {
     constexpr int M = N * N + 2 * N;
     __shared__ float cs[2 * M];
+    pdl_wait();
     for (int q = threadIdx.x; q < 2 * M; q += blockDim.x) {
         float a = 0.f;
         for (int p = 0; p < parts; ++p) a += part[(int64_t)p * 2 * M + q];
@@ -476,33 +483,43 @@ cudaError_t launch_n(const BwdArgs& a, const BwdLayout& L) {
         int64_t blocks = (Tn * 32 + RED_THREADS - 1) / RED_THREADS;
         const int64_t cap = (int64_t)di.sm_count * 8;
         if (blocks > cap) blocks = cap;
-        bwd_reduce_kernel<N, T><<<(unsigned)blocks, RED_THREADS, 0, a.stream>>>(
-            X, static_cast<const T*>(a.F), dY, dxi, a.H, Tn, d, R, static_cast<T*>(a.dF_out));
+        e = launch_pdl(bwd_reduce_kernel<N, T>, dim3((unsigned)blocks), dim3(RED_THREADS), 0, a.stream, X,
+                       static_cast<const T*>(a.F), dY, dxi, a.H, Tn, d, R, static_cast<T*>(a.dF_out));
+        if (e != cudaSuccess) return e;
     }
     unsigned char* rec = L.tc ? reinterpret_cast<unsigned char*>(ws + L.off_rec) : nullptr;
     const int64_t tok_threads = L.tc ? (Tn + BWD_REC_TILE - 1) / BWD_REC_TILE * BWD_REC_TILE : Tn;
-    bwd_token_kernel<N><<<(unsigned)((tok_threads + TOK_THREADS - 1) / TOK_THREADS), TOK_THREADS, 0, a.stream>>>(
-        R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res, Tn, K, a.eps, a.t_max, dl, G, beta, rec);
+    e = launch_pdl(bwd_token_kernel<N>, dim3((unsigned)((tok_threads + TOK_THREADS - 1) / TOK_THREADS)),
+                   dim3(TOK_THREADS), 0, a.stream, (const float*)R, a.H, a.h, a.b_res, a.a_pre, a.a_post, a.a_res,
+                   Tn, K, a.eps, a.t_max, dl, G, beta, rec);
+    if (e != cudaSuccess) return e;
     if (L.tc) {
         e = launch_bwd_tc(a, rec, part, L.groups, L.tokens_per_group);
         if (e != cudaSuccess) return e;
     } else {
         const int cs = dx_slice(N);
         dim3 grid((unsigned)((d + cs - 1) / cs), (unsigned)L.groups);
-        bwd_dx_dphi_kernel<N, T><<<grid, DX_THREADS, 0, a.stream>>>(
-            X, dY, dxi, a.phi, a.H, G, beta, Tn, d, L.tokens_per_group, static_cast<T*>(a.dX), part);
+        e = launch_pdl(bwd_dx_dphi_kernel<N, T>, grid, dim3(DX_THREADS), 0, a.stream, X, dY, dxi, a.phi, a.H,
+                       (const float*)G, (const float*)beta, Tn, d, (int)L.tokens_per_group, static_cast<T*>(a.dX),
+                       part);
+        if (e != cudaSuccess) return e;
     }
     {
         const int64_t len = (int64_t)K * M;
         int64_t blocks = (len + SUM_THREADS - 1) / SUM_THREADS;
         if (blocks > (int64_t)di.sm_count * 8) blocks = (int64_t)di.sm_count * 8;
-        bwd_dphi_sum_kernel<<<(unsigned)blocks, SUM_THREADS, 0, a.stream>>>(part, len, L.groups, a.dphi);
+        e = launch_pdl(bwd_dphi_sum_kernel, dim3((unsigned)blocks), dim3(SUM_THREADS), 0, a.stream,
+                       (const float*)part, len, L.groups, a.dphi);
+        if (e != cudaSuccess) return e;
     }
     {
         const int64_t per = (Tn + CS_PARTS - 1) / CS_PARTS;
-        bwd_colsum_part_kernel<M><<<CS_PARTS, SUM_THREADS, 0, a.stream>>>(dl, a.h, Tn, per, colsum);
-        bwd_colsum_final_kernel<N><<<1, 64, 0, a.stream>>>(colsum, CS_PARTS, a.db_pre, a.db_post, a.db_res,
-                                                           a.dalpha);
+        e = launch_pdl(bwd_colsum_part_kernel<M>, dim3(CS_PARTS), dim3(SUM_THREADS), 0, a.stream,
+                       (const float*)dl, a.h, Tn, per, colsum);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(bwd_colsum_final_kernel<N>, dim3(1), dim3(64), 0, a.stream, (const float*)colsum,
+                       (int)CS_PARTS, a.db_pre, a.db_post, a.db_res, a.dalpha);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

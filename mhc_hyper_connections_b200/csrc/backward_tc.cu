@@ -286,6 +286,7 @@ bwd_tc_kernel(const __grid_constant__ Maps maps, const float* __restrict__ phi,
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_slot;
+    pdl_wait();                 // the token records are the previous kernel's; everything above is not
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -568,10 +569,9 @@ cudaError_t launch_n(const BwdArgs& a, const void* rec, float* part, int groups,
     }
     const int slices = a.d / CW;
     const unsigned grid = (unsigned)(slices * groups);
-    bwd_tc_kernel<N><<<grid, THREADS, Cfg<N>::SMEM, a.stream>>>(
-        maps, a.phi, static_cast<const unsigned char*>(rec), (int)a.T, a.d, (int)tpg,
-        static_cast<__nv_bfloat16*>(a.dX), part, g_stop_stage.load(), g_wait_ns.load());
-    return cudaGetLastError();
+    return launch_pdl(bwd_tc_kernel<N>, dim3(grid), dim3(THREADS), (size_t)Cfg<N>::SMEM, a.stream, maps, a.phi,
+                      static_cast<const unsigned char*>(rec), (int)a.T, a.d, (int)tpg,
+                      static_cast<__nv_bfloat16*>(a.dX), part, g_stop_stage.load(), g_wait_ns.load());
 }
 
 }  // namespace bwdtc

@@ -71,6 +71,29 @@ cudaError_t pre_wide_status(unsigned* out, bool clear);
 
 cudaError_t launch_post(const PostArgs& a);
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel on the stream finishes; it must execute pdl_wait() before it reads or writes any
+// memory the previous work touches (without the attribute pdl_wait is a no-op).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+// wait for the previous kernel on the stream to complete and its memory to be visible
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// let the next kernel on the stream (launched with launch_pdl) start its own prologue
+__device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Reverse mode of pre + post (backward.cu).
 struct BwdArgs {
     const void* X;
