@@ -46,13 +46,13 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum per launch, captured at half the token count
     # (X still twice the L2) and scaled x2 (profiles/ holds the commands and the raw counts)
     ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.129920 + 41.285632) * 2e6), "157c4df346643206"),
-    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.353792 + 209.392128) * 2e6), "96dbcd70460419e6"),
+    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.344576 + 210.202112) * 2e6), "0a821a0f07264b90"),
     # the three launches of the two-pass path at T=4096: the projection and read-map kernels
     # scaled x2, the phi packing (no token dependence) once
     ("pre", "bf16_T8192_n8_d4096"): (int(((279.553280 + 0.129280 + 268.969728 + 6.182144) * 2 + 10.491392) * 1e6),
                                      "a3245bd1e65cf5b5"),
     # the six launches of one mhc_backward call at T=8192, scaled x2 (backward.cu + backward_tc.cu)
-    ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.784 + 252.221184) * 2e6), "886ee410090ef055"),
+    ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.79808 + 249.99424) * 2e6), "49ace6afacd92d5a"),
 }
 
 
