@@ -110,13 +110,16 @@ def make_inputs(T: int, n: int, d: int, dtype: str = "bf16", seed: int = 0,
                     alpha_post=alpha, alpha_res=alpha, outlier_channels=ch)
 
 
-# The four forward workloads: sizes, storage type, seed and outlier structure.
+# The four forward workloads (and one extra shape): sizes, storage type, seed and outlier structure.
 CONFIGS = {
     "tiny_f32_T64_n4_d64": dict(T=64, n=4, d=64, dtype="f32", seed=0),
     "bf16_T4096_n4_d1024": dict(T=4096, n=4, d=1024, dtype="bf16", seed=1),
     "bf16_T16384_n4_d4096_outliers": dict(T=16384, n=4, d=4096, dtype="bf16", seed=2,
                                           outlier_frac=0.01),
     "bf16_T8192_n8_d4096": dict(T=8192, n=8, d=4096, dtype="bf16", seed=3),
+    # not one of the four: the hidden size of the 27B model in the "DeepSeek-V4/mhc" model
+    # table, for a bench figure of that shape
+    "bf16_T16384_n4_d2560": dict(T=16384, n=4, d=2560, dtype="bf16", seed=4),
 }
 
 HEADLINE = "bf16_T16384_n4_d4096_outliers"
