@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum per launch, captured at half the token count
     # (X still twice the L2) and scaled x2 (profiles/ holds the commands and the raw counts)
-    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.129920 + 41.285632) * 2e6), "157c4df346643206"),
+    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.201600 + 41.880064) * 2e6), "b2019263f3ba751a"),
     ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.344576 + 210.202112) * 2e6), "0a821a0f07264b90"),
     # the three launches of the two-pass path at T=4096: the projection and read-map kernels
     # scaled x2, the phi packing (no token dependence) once
