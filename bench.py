@@ -403,7 +403,9 @@ def run_ours(args, rank, world, local_rank):
            "frac_of_measured": step_gbs / peak,
            "frac_of_8TBs_lit": (2 * n + 2) * d * es * T / (ms_total / 1e3 / K) / 1e9 / NOMINAL_HBM_GBS}
 
-    # ---- end to end through the public API with host buffers (pinned), copies timed
+    # ---- end to end through the public API with host buffers (pinned), copies timed: one
+    # mhc_forward_host call per step, which copies each chunk of tokens in, runs pre and post on
+    # it and copies its outputs back, overlapping the two copy directions and the kernels
     e2e = None
     if not args.no_e2e:
         Ke = max(1, min(K, args.e2e_steps))
@@ -414,15 +416,14 @@ def run_ours(args, rank, world, local_rank):
         xo = torch.empty_like(x_in, device="cpu").pin_memory()
         Ho = torch.empty_like(H, device="cpu").pin_memory()
         Yo = torch.empty_like(Y, device="cpu").pin_memory()
+        chunk = min(args.e2e_chunk, T)
+        ws_e2e = torch.empty(mhc.mhc_forward_host_workspace_bytes(chunk, n, d, X.dtype),
+                             dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            X.copy_(Xh, non_blocking=True)
-            F.copy_(Fh, non_blocking=True)
-            pre()
-            post()
-            xo.copy_(x_in, non_blocking=True)
-            Ho.copy_(H, non_blocking=True)
-            Yo.copy_(Y, non_blocking=True)
+            mhc.mhc_forward_host(Xh, Fh, phi, b_pre, b_post, b_res, s["alpha_pre"], s["alpha_post"],
+                                 s["alpha_res"], s["eps"], s["t_max"], xo, Ho, Yo, ws_e2e,
+                                 chunk_tokens=chunk)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -438,7 +439,8 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": mdist.job_throughput(T, Ke, e_ms, world), "unit": "tokens/s",
                "h2d_bytes_per_step": (X.numel() + F.numel()) * es,
                "d2h_bytes_per_step": (x_in.numel() * es + H.numel() * 4 + Y.numel() * es),
-               "steps": Ke}
+               "steps": Ke, "api": "mhc_forward_host (pre path auto)", "chunk_tokens": chunk}
+        del ws_e2e
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -659,6 +661,8 @@ def main():
                     help="kernel path of the pre stage (default: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-chunk", type=int, default=1024,
+                    help="tokens per chunk of the end-to-end mhc_forward_host call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--amax", action="store_true",

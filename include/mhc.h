@@ -20,11 +20,12 @@
  *     section "Details van de parameterisatie": H_pre in (0,1), H_post in (0,2).
  *
  * Conventions shared by every entry point
- *   - All data pointers are DEVICE pointers.  The caller allocates and owns every
+ *   - All data pointers are DEVICE pointers, except the activations of
+ *     mhc_forward_host, which live in host memory.  The caller allocates and owns every
  *     buffer; the library allocates no device memory.  Between calls it keeps a
- *     per-device cache of kernel launch limits and, in its device image, the status
- *     word of the bounded waits (mhc_device_status) and the fixed scratch array of
- *     mhc_backward_noalloc.
+ *     per-device cache of kernel launch limits, the two copy streams of
+ *     mhc_forward_host and, in its device image, the status word of the bounded waits
+ *     (mhc_device_status) and the fixed scratch array of mhc_backward_noalloc.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Arguments are validated on the host before any launch; a rejected
  *     call launches nothing and returns a non-zero mhc_status.  MHC_ERR_CUDA means
@@ -72,7 +73,7 @@ typedef enum {
     MHC_ERR_UNSUPPORTED = 5,   /* the requested kernel path cannot run this problem  */
     MHC_ERR_CUDA = 6,          /* a CUDA call or launch failed                       */
     MHC_ERR_ALIAS = 7,         /* an output overlaps an input or another output      */
-    MHC_ERR_WORKSPACE = 8      /* workspace smaller than mhc_backward_workspace_bytes */
+    MHC_ERR_WORKSPACE = 8      /* workspace smaller than its *_workspace_bytes query  */
 } mhc_status;
 
 typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
@@ -167,6 +168,46 @@ int mhc_pre_path_ok(int64_t T, int n, int d, mhc_dtype dt, mhc_pre_path path);
  */
 mhc_status mhc_post(const void* X, const void* F_out, const float* H, int64_t T, int n, int d,
                     mhc_dtype dt, void* X_out, mhc_stream_t stream);
+
+/*
+ * mhc_forward_host -- mhc_pre, then mhc_post, for T tokens whose activations live in HOST
+ * memory (slavadubrov.com Eq. 3 with the sub-layer's output F_out given, as mhc_post takes
+ * it).  This is the one entry point with host pointers:
+ *   host   : X_h [T,n,d], F_out_h [T,d] (inputs); x_in_h [T,d], H_h [T,m], X_out_h [T,n,d]
+ *            (outputs), same layouts and dtypes as the device entry points.  Page-locked
+ *            (pinned) host memory lets the copies overlap; pageable memory gives the same
+ *            results with the copies serialised by the driver.
+ *   device : phi, b_pre, b_post, b_res (the parameters stay resident on the device), and
+ *            `workspace`, 256-byte aligned, at least
+ *            mhc_forward_host_workspace_bytes(chunk_tokens, n, d, dt) bytes.  It may not
+ *            overlap the parameters.
+ * The tokens go through in chunks of chunk_tokens (the last chunk may be shorter), rotating
+ * through three device buffer sets in the workspace. The copies into the device of chunk c+1,
+ * the two stages on chunk c and the copies back of chunk c-1 overlap. The copies use two
+ * streams of the library's own, created on the first call on a device and kept for the
+ * process. Everything is ordered after the work already queued on `stream`, and `stream`
+ * resumes only once every output has landed in host memory. So a host read of the outputs
+ * needs a synchronisation of `stream`, and the workspace may be reused by the next call on
+ * the same stream.
+ * Every output of a token depends on that token alone, so the outputs are those of mhc_pre
+ * and mhc_post called on each chunk. That is bit for bit the whole-batch result wherever the
+ * chunk takes the same kernel path (mhc_pre_path_for).
+ * Errors: the argument checks of mhc_pre, plus MHC_ERR_SHAPE for chunk_tokens < 1 (or a
+ * chunk too large to address), MHC_ERR_WORKSPACE, and MHC_ERR_ALIAS for host outputs that
+ * overlap a host input or each other, or a workspace that overlaps the parameters.  All of
+ * them are checked before anything is queued.  A CUDA failure part-way (MHC_ERR_CUDA) leaves
+ * the outputs incomplete, and copies already queued may still run: synchronise the device
+ * before reusing the host buffers.  Calls on one device from several host threads are
+ * serialised while they queue their work.
+ */
+size_t mhc_forward_host_workspace_bytes(int64_t chunk_tokens, int n, int d, mhc_dtype dt);
+
+mhc_status mhc_forward_host(const void* X_h, const void* F_out_h, const float* phi,
+                            const float* b_pre, const float* b_post, const float* b_res,
+                            float alpha_pre, float alpha_post, float alpha_res, int64_t T, int n,
+                            int d, float eps, int t_max, mhc_dtype dt, void* x_in_h, float* H_h,
+                            void* X_out_h, int64_t chunk_tokens, void* workspace,
+                            size_t workspace_bytes, mhc_stream_t stream);
 
 /*
  * mhc_pre_train -- mhc_pre for training: the same computation and outputs, plus the

@@ -27,7 +27,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_post", "mhc_backward",
+__all__ = ["mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_post",
+           "mhc_forward_host", "mhc_forward_host_workspace_bytes", "mhc_backward",
            "mhc_backward_workspace_bytes", "mhc_backward_noalloc", "NOALLOC_SCRATCH_BYTES",
            "mhc_amax_gain", "mhc_pre_path_for", "mhc_pre_path_ok", "mhc_device_status",
            "mhc_debug_pre_stop_after", "mhc_debug_backward_stop_after",
@@ -47,7 +48,7 @@ _STATUS = {0: "MHC_OK", 1: "MHC_ERR_NULL", 2: "MHC_ERR_SHAPE", 3: "MHC_ERR_ALIGN
 
 # Every function include/mhc.h declares.
 EXPORTED_SYMBOLS = ("mhc_pre", "mhc_pre_with_path", "mhc_pre_hc", "mhc_pre_train", "mhc_pre_path_for",
-                    "mhc_pre_path_ok", "mhc_post",
+                    "mhc_pre_path_ok", "mhc_post", "mhc_forward_host_workspace_bytes", "mhc_forward_host",
                     "mhc_backward_workspace_bytes", "mhc_backward", "mhc_backward_noalloc",
                     "mhc_amax_gain", "mhc_status_string",
                     "mhc_last_error", "mhc_device_status", "mhc_debug_pre_stop_after",
@@ -104,6 +105,11 @@ def load_library():
         lib.mhc_pre_path_ok.restype = ci
         lib.mhc_post.argtypes = [vp, vp, fp, i64, ci, ci, ci, vp, vp]
         lib.mhc_post.restype = ci
+        lib.mhc_forward_host_workspace_bytes.argtypes = [i64, ci, ci, ci]
+        lib.mhc_forward_host_workspace_bytes.restype = ctypes.c_size_t
+        lib.mhc_forward_host.argtypes = ([vp, vp, fp, fp, fp, fp, cf, cf, cf, i64, ci, ci, cf, ci, ci,
+                                          vp, fp, vp, i64, vp, ctypes.c_size_t, vp])
+        lib.mhc_forward_host.restype = ci
         lib.mhc_status_string.argtypes = [ci]
         lib.mhc_status_string.restype = ctypes.c_char_p
         lib.mhc_last_error.argtypes = []
@@ -241,6 +247,64 @@ def mhc_post(X, F_out, H, X_out, stream=None):
     with torch.cuda.device(dev):
         st = lib.mhc_post(px, pf, ph, T, n, d, _dt(X), po, _stream(stream, dev))
     _check(st, "mhc_post")
+
+
+def _host_ptr(t, name, dtype=None) -> int:
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch tensor in host memory")
+    if t.is_cuda:
+        raise ValueError(f"{name}: must be a host (CPU) tensor; pinned memory lets the copies overlap")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def mhc_forward_host_workspace_bytes(chunk_tokens: int, n: int, d: int, dtype) -> int:
+    """Device workspace bytes mhc_forward_host needs for chunks of chunk_tokens tokens."""
+    import torch
+    dt = MHC_BF16 if dtype == torch.bfloat16 else MHC_F32 if dtype == torch.float32 else None
+    if dt is None:
+        raise TypeError(f"unsupported dtype {dtype}")
+    v = load_library().mhc_forward_host_workspace_bytes(int(chunk_tokens), int(n), int(d), dt)
+    if v == 0:
+        raise MhcError(2, "mhc_forward_host_workspace_bytes", "chunk_tokens, n or d out of range")
+    return v
+
+
+def mhc_forward_host(X_h, F_out_h, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res,
+                     eps, t_max, x_in_h, H_h, X_out_h, workspace, chunk_tokens: int = 1024,
+                     stream=None):
+    """mhc_pre then mhc_post on activations in host memory (X_h [T, n, d], F_out_h [T, d];
+    outputs x_in_h [T, d], H_h [T, m], X_out_h [T, n, d], all CPU tensors, pinned for overlap).
+    The parameters and the uint8 workspace (mhc_forward_host_workspace_bytes) are CUDA tensors.
+    Asynchronous on `stream`: synchronise it before reading the outputs."""
+    import torch
+    T, n, d = X_h.shape
+    m = n * n + 2 * n
+    dev = phi.device
+    f32 = torch.float32
+    if tuple(F_out_h.shape) != (T, d) or tuple(x_in_h.shape) != (T, d) or tuple(H_h.shape) != (T, m) \
+            or tuple(X_out_h.shape) != (T, n, d) or tuple(phi.shape) != (n * d, m):
+        raise ValueError("mhc_forward_host: shapes must be F_out_h, x_in_h [T, d], H_h [T, m], "
+                         "X_out_h [T, n, d], phi [n*d, m]")
+    if b_pre.numel() != n or b_post.numel() != n or b_res.numel() != n * n:
+        raise ValueError("mhc_forward_host: b_pre/b_post need n entries, b_res n*n")
+    hp = dict(X=_host_ptr(X_h, "X_h"), F=_host_ptr(F_out_h, "F_out_h", X_h.dtype),
+              xin=_host_ptr(x_in_h, "x_in_h", X_h.dtype), H=_host_ptr(H_h, "H_h", f32),
+              Y=_host_ptr(X_out_h, "X_out_h", X_h.dtype))
+    dp = dict(phi=_ptr(phi, "phi", f32, dev), b_pre=_ptr(b_pre, "b_pre", f32, dev),
+              b_post=_ptr(b_post, "b_post", f32, dev), b_res=_ptr(b_res, "b_res", f32, dev),
+              ws=_ptr(workspace, "workspace", torch.uint8, dev))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.mhc_forward_host(hp["X"], hp["F"], dp["phi"], dp["b_pre"], dp["b_post"], dp["b_res"],
+                                  float(alpha_pre), float(alpha_post), float(alpha_res), T, n, d,
+                                  float(eps), int(t_max), _dt(X_h), hp["xin"], hp["H"], hp["Y"],
+                                  int(chunk_tokens), dp["ws"], workspace.numel(), _stream(stream, dev))
+    _check(st, "mhc_forward_host")
 
 
 def mhc_pre_train(X, phi, b_pre, b_post, b_res, alpha_pre, alpha_post, alpha_res, eps, t_max,

@@ -333,7 +333,7 @@ const char* mhc_status_string(mhc_status s) {
         case MHC_ERR_UNSUPPORTED: return "the requested kernel path cannot run this problem";
         case MHC_ERR_CUDA: return "a CUDA call or launch failed (see mhc_last_error)";
         case MHC_ERR_ALIAS: return "an output overlaps an input or another output";
-        case MHC_ERR_WORKSPACE: return "the workspace is smaller than mhc_backward_workspace_bytes";
+        case MHC_ERR_WORKSPACE: return "the workspace is smaller than its *_workspace_bytes query";
     }
     return "unknown status";
 }

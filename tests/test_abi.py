@@ -87,6 +87,39 @@ def test_post_validation(lib):
     assert post(Y=A + 0x1000000) == 7                # X_out overlaps F_out
 
 
+def test_forward_host_validation(lib):
+    """mhc_forward_host: every rejection happens before the library touches CUDA."""
+    n, d, T, ct = 4, 64, 10, 4
+    ws_need = lib.mhc_forward_host_workspace_bytes(ct, n, d, 1)
+    assert ws_need > 0
+    assert lib.mhc_forward_host_workspace_bytes(2 * ct, n, d, 1) > ws_need
+    assert lib.mhc_forward_host_workspace_bytes(0, n, d, 1) == 0
+    assert lib.mhc_forward_host_workspace_bytes(ct, 9, d, 1) == 0
+    assert lib.mhc_forward_host_workspace_bytes(ct, n, d, 5) == 0
+    assert lib.mhc_forward_host_workspace_bytes(1 << 40, n, d, 1) == 0   # a chunk too large
+
+    W = A + 0x5000000                                # device workspace (256-aligned)
+
+    def fh(Xh=A, Fh=A + 0x1000000, phi=A + 0x6000000, bp=A + 0x7000000, bq=A + 0x7000100,
+           br=A + 0x7000200, T=T, n=n, d=d, t_max=20, dt=1, xin=A + 0x2000000, Hh=A + 0x3000000,
+           Yh=A + 0x4000000, ct=ct, ws=W, wsb=ws_need):
+        return lib.mhc_forward_host(Xh, Fh, phi, bp, bq, br, 0.01, 0.01, 0.01, T, n, d, 1e-20,
+                                    t_max, dt, xin, Hh, Yh, ct, ws, wsb, None)
+    assert fh(T=0) == 0 and fh(T=0, Xh=0, ws=0) == 0   # no tokens: nothing to do
+    assert fh(n=9) == 2 and fh(d=0) == 2 and fh(t_max=1001) == 2
+    assert fh(ct=0) == 2 and fh(ct=-5) == 2
+    assert fh(dt=3) == 4
+    assert fh(Xh=0) == 1 and fh(Yh=0) == 1 and fh(ws=0) == 1 and fh(br=0) == 1
+    assert fh(Xh=A + 1) == 3 and fh(Hh=A + 0x3000002) == 3
+    assert fh(ws=W + 16) == 3                        # the workspace needs 256-byte alignment
+    assert fh(wsb=ws_need - 1) == 8
+    assert fh(ct=100) == 8                           # a chunk above T takes all T = 10 tokens
+    assert fh(xin=A + 64) == 7                       # x_in_h overlaps X_h
+    assert fh(Yh=A + 0x1000000) == 7                 # X_out_h overlaps F_out_h
+    assert fh(Hh=A + 0x2000000) == 7                 # H_h overlaps x_in_h
+    assert fh(phi=W + 256) == 7                      # the workspace holds phi
+
+
 def test_binding_refuses_host_tensors():
     torch = pytest.importorskip("torch")
     X = torch.zeros(2, 4, 8, dtype=torch.bfloat16)
