@@ -43,12 +43,42 @@ constexpr int SUM_THREADS = 256;
 __host__ __device__ constexpr int red_len(int n) { return 1 + n + n * n + n; }
 
 // ---------------------------------------------------------------- K1
+// Element pairs of a 16-byte word as float2 (2p, 2p + 1), for the paired FMAs below.
+template <typename T> struct Pairs;
+template <> struct Pairs<__nv_bfloat16> {
+    static constexpr int NP = 4;
+    __device__ __forceinline__ static float2 get(const uint4& w, int p) {
+        return bf16x2_to_f32x2(p == 0 ? w.x : p == 1 ? w.y : p == 2 ? w.z : w.w);
+    }
+    // rounds the pair to bf16 into word p
+    __device__ __forceinline__ static void put(uint4& w, int p, float2 v) {
+        const uint32_t u = pack_bf16x2(v.x, v.y);
+        if (p == 0) w.x = u; else if (p == 1) w.y = u; else if (p == 2) w.z = u; else w.w = u;
+    }
+};
+template <> struct Pairs<float> {
+    static constexpr int NP = 2;
+    __device__ __forceinline__ static float2 get(const uint4& w, int p) {
+        return p == 0 ? make_float2(__uint_as_float(w.x), __uint_as_float(w.y))
+                      : make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+    }
+    __device__ __forceinline__ static void put(uint4& w, int p, float2 v) {
+        if (p == 0) { w.x = __float_as_uint(v.x); w.y = __float_as_uint(v.y); }
+        else { w.z = __float_as_uint(v.x); w.w = __float_as_uint(v.y); }
+    }
+};
+
+// One warp per token: the token's reductions R (sum of squares, dx_in . X_i, dX_out_i . X_j,
+// dX_out_i . F_out) and dF_out = sum_i H_post[i] dX_out_i.  Each lane walks 16-byte chunks of
+// the d channels; its sums run over even and odd channels separately (packed fp32x2 FMAs) and
+// are added at the end, then across the warp in a fixed order.
 template <int N, typename T>
-__global__ void __launch_bounds__(RED_THREADS)
+__global__ void __launch_bounds__(RED_THREADS, 2)
 bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __restrict__ dY,
                   const T* __restrict__ dx, const float* __restrict__ H, int64_t Tn, int d,
                   float* __restrict__ R, T* __restrict__ dF) {
     constexpr int M = N * N + 2 * N, NR = red_len(N), V = Vec16<T>::VEC;
+    using P = Pairs<T>;
     const int lane = threadIdx.x & 31;
     pdl_wait();
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -57,50 +87,54 @@ bwd_reduce_kernel(const T* __restrict__ X, const T* __restrict__ F, const T* __r
         float hpost[N];
 #pragma unroll
         for (int i = 0; i < N; ++i) hpost[i] = __ldg(H + t * M + N + N * N + i);
-        float acc[NR];
+        float2 acc[NR];
 #pragma unroll
-        for (int q = 0; q < NR; ++q) acc[q] = 0.f;
+        for (int q = 0; q < NR; ++q) acc[q] = make_float2(0.f, 0.f);
         for (int q = lane; q < nchunk; q += 32) {
-            float fx[N][V], fd[V], ff[V], df[V];
+            uint4 wx[N], wy[N];
 #pragma unroll
-            for (int i = 0; i < N; ++i) Vec16<T>::unpack(ld_stream_v4(X + (t * N + i) * d + q * V), fx[i]);
-            Vec16<T>::unpack(ld_stream_v4(dx + t * d + q * V), fd);
-            Vec16<T>::unpack(ld_stream_v4(F + t * d + q * V), ff);
+            for (int i = 0; i < N; ++i) wx[i] = ld_stream_v4(X + (t * N + i) * d + q * V);
+            const uint4 wd = ld_stream_v4(dx + t * d + q * V);
+            const uint4 wf = ld_stream_v4(F + t * d + q * V);
 #pragma unroll
-            for (int e = 0; e < V; ++e) df[e] = 0.f;
+            for (int i = 0; i < N; ++i) wy[i] = ld_stream_v4(dY + (t * N + i) * d + q * V);
+            uint4 dfw;
 #pragma unroll
-            for (int i = 0; i < N; ++i) {
+            for (int p = 0; p < P::NP; ++p) {
+                float2 x[N];
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    acc[0] = fmaf(fx[i][e], fx[i][e], acc[0]);
-                    acc[1 + i] = fmaf(fd[e], fx[i][e], acc[1 + i]);
+                for (int i = 0; i < N; ++i) x[i] = P::get(wx[i], p);
+                const float2 dv = P::get(wd, p), fv = P::get(wf, p);
+#pragma unroll
+                for (int i = 0; i < N; ++i) {
+                    acc[0] = __ffma2_rn(x[i], x[i], acc[0]);
+                    acc[1 + i] = __ffma2_rn(dv, x[i], acc[1 + i]);
                 }
-            }
+                float2 dfp = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < N; ++i) {
-                float fy[V];
-                Vec16<T>::unpack(ld_stream_v4(dY + (t * N + i) * d + q * V), fy);
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    acc[1 + N + N * N + i] = fmaf(fy[e], ff[e], acc[1 + N + N * N + i]);
-                    df[e] = fmaf(hpost[i], fy[e], df[e]);
+                for (int i = 0; i < N; ++i) {
+                    const float2 y = P::get(wy[i], p);
+                    acc[1 + N + N * N + i] = __ffma2_rn(y, fv, acc[1 + N + N * N + i]);
+                    dfp = __ffma2_rn(make_float2(hpost[i], hpost[i]), y, dfp);
 #pragma unroll
                     for (int j = 0; j < N; ++j)
-                        acc[1 + N + i * N + j] = fmaf(fy[e], fx[j][e], acc[1 + N + i * N + j]);
+                        acc[1 + N + i * N + j] = __ffma2_rn(y, x[j], acc[1 + N + i * N + j]);
                 }
+                P::put(dfw, p, dfp);
             }
-            st_v4(dF + t * d + q * V, Vec16<T>::pack(df));
+            st_v4(dF + t * d + q * V, dfw);
         }
+        float red[NR];
 #pragma unroll
         for (int q = 0; q < NR; ++q) {
-            float v = acc[q];
+            float v = acc[q].x + acc[q].y;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-            acc[q] = v;
+            red[q] = v;
         }
 #pragma unroll
         for (int q = 0; q < NR; ++q)
-            if (lane == (q & 31)) R[t * NR + q] = acc[q];
+            if (lane == (q & 31)) R[t * NR + q] = red[q];
     }
 }
 
