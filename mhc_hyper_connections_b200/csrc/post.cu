@@ -48,6 +48,9 @@ __device__ __forceinline__ void load_coeffs(const float* __restrict__ Ht, float 
     }
 }
 
+// Launched plainly, after the previous work on the stream has finished: with a programmatic
+// dependent launch (griddepcontrol.wait at the top) the n = 8 instance compiled to 182 registers
+// instead of 128 and streamed at 70 % of the copy bandwidth instead of 90 %.
 template <int N, typename T, bool HV>
 __global__ void __launch_bounds__(THREADS)
 post_vec_kernel(const T* __restrict__ X, const T* __restrict__ F, const float* __restrict__ H,
@@ -58,7 +61,6 @@ post_vec_kernel(const T* __restrict__ X, const T* __restrict__ F, const float* _
     const int chunks = d / VEC;
     const int tasks_per_tok = (chunks + 31) >> 5;
     const int64_t ntasks = Tn * tasks_per_tok;
-    pdl_wait();                 // X, F_out and H are the previous work's
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t task = (((int64_t)blockIdx.x * blockDim.x) + threadIdx.x) >> 5; task < ntasks;
@@ -102,7 +104,6 @@ post_scalar_kernel(const T* __restrict__ X, const T* __restrict__ F, const float
     constexpr int M = N * N + 2 * N;
     const int64_t total = Tn * d;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    pdl_wait();
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
         const int64_t t = e / d;
         const int c = (int)(e - t * d);
@@ -140,17 +141,14 @@ cudaError_t launch_n(const PostArgs& a) {
         const int64_t want = (tasks * 32 + THREADS - 1) / THREADS;
         const int64_t cap = (int64_t)di.sm_count * (per_sm > 0 ? per_sm : 1);
         const unsigned blocks = (unsigned)(want < cap ? want : cap);
-        e = launch_pdl(kern, dim3(blocks), dim3(THREADS), 0, a.stream, static_cast<const T*>(a.X),
-                       static_cast<const T*>(a.F), a.H, a.T, a.d, static_cast<T*>(a.Y));
-        if (e != cudaSuccess) return e;
+        kern<<<blocks, THREADS, 0, a.stream>>>(static_cast<const T*>(a.X), static_cast<const T*>(a.F), a.H,
+                                                a.T, a.d, static_cast<T*>(a.Y));
     } else {
         const int64_t want = (a.T * a.d + THREADS - 1) / THREADS;
         const int64_t cap = (int64_t)di.sm_count * 8;
         const unsigned blocks = (unsigned)(want < cap ? want : cap);
-        e = launch_pdl(post_scalar_kernel<N, T>, dim3(blocks), dim3(THREADS), 0, a.stream,
-                       static_cast<const T*>(a.X), static_cast<const T*>(a.F), a.H, a.T, a.d,
-                       static_cast<T*>(a.Y));
-        if (e != cudaSuccess) return e;
+        post_scalar_kernel<N, T><<<blocks, THREADS, 0, a.stream>>>(
+            static_cast<const T*>(a.X), static_cast<const T*>(a.F), a.H, a.T, a.d, static_cast<T*>(a.Y));
     }
     return cudaGetLastError();
 }

@@ -196,7 +196,7 @@ __device__ __forceinline__ void owner_maps4(const float* hv, float inv_r, int gl
 #pragma unroll
             for (int j = 0; j < N; ++j) cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 2);
 #pragma unroll
-            for (int j = 0; j < N; ++j) cs[j] = 1.0f / cs[j];
+            for (int j = 0; j < N; ++j) cs[j] = __fdividef(1.0f, cs[j]);
 #pragma unroll
             for (int j = 0; j < N; ++j) {
                 Mx[0][j] *= cs[j];
@@ -208,7 +208,7 @@ __device__ __forceinline__ void owner_maps4(const float* hv, float inv_r, int gl
                 float s = 0.f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) s += Mx[r][j];
-                rs[r] = own[r] ? 1.0f / s : 0.f;
+                rs[r] = own[r] ? __fdividef(1.0f, s) : 0.f;
             }
 #pragma unroll
             for (int r = 0; r < 2; ++r)
