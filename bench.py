@@ -45,14 +45,14 @@ FALLBACK_HBM_GBS = 6650.0         # used only if MEASURED_PEAKS.json is absent
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum per launch, captured at half the token count
     # (X still twice the L2) and scaled x2 (profiles/ holds the commands and the raw counts)
-    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.201600 + 41.880064) * 2e6), "b2019263f3ba751a"),
-    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.344576 + 210.202112) * 2e6), "0a821a0f07264b90"),
+    ("pre", "bf16_T16384_n4_d4096_outliers"): (int((270.448128 + 41.708544) * 2e6), "b2019263f3ba751a"),
+    ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.344832 + 210.074368) * 2e6), "e2d0eca830bf798b"),
     # the three launches of the two-pass path at T=4096: the projection and read-map kernels
     # scaled x2, the phi packing (no token dependence) once
-    ("pre", "bf16_T8192_n8_d4096"): (int(((279.553280 + 0.129280 + 268.969728 + 6.182144) * 2 + 10.491392) * 1e6),
-                                     "a3245bd1e65cf5b5"),
+    ("pre", "bf16_T8192_n8_d4096"): (int(((279.602432 + 0.499200 + 268.970752 + 6.845440) * 2 + 10.491136) * 1e6),
+                                     "0dfa0d4015ab4244"),
     # the six launches of one mhc_backward call at T=8192, scaled x2 (backward.cu + backward_tc.cu)
-    ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.79808 + 249.99424) * 2e6), "49ace6afacd92d5a"),
+    ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.790400 + 261.519104) * 2e6), "bab5f002ab08645e"),
 }
 
 
