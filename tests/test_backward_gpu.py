@@ -120,11 +120,13 @@ def test_bf16_d1024_full():
 @pytest.mark.parametrize("T,n,d,dt", [(1, 1, 8, "bf16"), (33, 2, 24, "f32"), (100, 3, 136, "bf16"),
                                       (37, 4, 64, "bf16"), (300, 1, 1024, "bf16"), (65, 3, 12, "f32"),
                                       (129, 3, 192, "bf16"), (1000, 2, 640, "bf16"), (64, 4, 128, "bf16"),
-                                      (200, 4, 4096, "bf16"), (1, 2, 64, "bf16"), (777, 1, 128, "bf16")])
+                                      (200, 4, 4096, "bf16"), (1, 2, 64, "bf16"), (777, 1, 128, "bf16"),
+                                      (64, 4, 12800, "bf16"), (100, 2, 9600, "bf16"), (50, 1, 25600, "bf16")])
 def test_shapes(T, n, d, dt):
     """Ragged shapes on both dX / dphi kernels: bf16 with d a multiple of 64 takes the
     tensor-core step (token tails inside a stage, groups that end mid-tensor or hold no
-    tokens, odd n with a placeholder stream), the rest the CUDA-core step."""
+    tokens, odd n with a placeholder stream, and wide d: 150 to 400 channel slices), the rest
+    the CUDA-core step."""
     w = wl.make_inputs(T=T, n=n, d=d, dtype=dt, seed=T * 7 + n * 3 + d, alpha=0.3)
     dY, dx = _upstream(w, T + d)
     check(w, run_gpu(w, dY, dx), run_oracle(w, dY, dx), f"T{T} n{n} d{d} {dt}")
