@@ -141,3 +141,35 @@ def test_forward_host_reuses_workspace_across_calls():
     r = (hb1["x_in"], hb1["H"], hb1["Y"], hb2["x_in"], hb2["H"], hb2["Y"])
     for x, y in zip(r, d1 + d2):
         assert torch.equal(_bits(x), _bits(y))
+
+
+def test_forward_host_two_host_threads():
+    """Two host threads call mhc_forward_host at once, each on its own stream and workspace:
+    the library's copy streams are shared, and each call still sees its own inputs."""
+    import threading
+    ws_ = [wl.make_inputs(T=700, n=4, d=1024, dtype="bf16", seed=16 + k) for k in range(2)]
+    ts = [torch_inputs(w) for w in ws_]
+    hbs = [_host_buffers(w, t) for w, t in zip(ws_, ts)]
+    wss = [_workspace(256, w, torch.bfloat16) for w in ws_]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    errors = []
+
+    def worker(k):
+        try:
+            with torch.cuda.stream(streams[k]):
+                for _ in range(3):
+                    _call(ws_[k], ts[k], hbs[k], 256, wss[k])
+            streams[k].synchronize()
+        except Exception as e:          # surfaced below
+            errors.append(e)
+    th = [threading.Thread(target=worker, args=(k,)) for k in range(2)]
+    for t_ in th:
+        t_.start()
+    for t_ in th:
+        t_.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    for k in range(2):
+        ref = _chunked_device(ws_[k], ts[k], 256)
+        for x, y in zip((hbs[k]["x_in"], hbs[k]["H"], hbs[k]["Y"]), ref):
+            assert torch.equal(_bits(x), _bits(y))
