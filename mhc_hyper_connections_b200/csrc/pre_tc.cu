@@ -68,8 +68,7 @@ constexpr int PF = 0;              // stages of X prefetched into L2 ahead of th
 constexpr int NXW = 7;             // x_in warps
 constexpr int SK_WARP = 8 + NXW;   // Sinkhorn warp
 constexpr int BATCH = 32;          // tokens per Sinkhorn pass (one per lane)
-constexpr int NPASS = 2;           // logit ring: passes
-constexpr int RING = NPASS * BATCH;
+constexpr int RING = 2 * BATCH;    // logit ring: two passes
 constexpr int XU = 2;              // x_in tasks in flight per thread (more slows the X stream: 5 took 7 % longer)
 constexpr int NWARPS = 16;         // 4 warps per scheduler partition: up to 128 registers
 constexpr int THREADS = NWARPS * 32;
@@ -106,7 +105,7 @@ enum : int {
     B_PFULL = B_ACCE + NACC, B_PEMPTY = B_PFULL + NSLOT_P, B_HFULL = B_PEMPTY + NSLOT_P,
     B_HEMPTY = B_HFULL + NSLOT_H, B_DRAIN = B_HEMPTY + NSLOT_H, B_STG_FREE = B_DRAIN + NMMA,
     B_STG_READY = B_STG_FREE + 2, B_XDONE = B_STG_READY + 1, B_LG_FULL = B_XDONE + NSLOT_H,
-    B_LG_EMPTY = B_LG_FULL + NPASS, B_COUNT = B_LG_EMPTY + NPASS
+    B_LG_EMPTY = B_LG_FULL + 2, B_COUNT = B_LG_EMPTY + 2
 };
 
 // status codes: which wait expired
@@ -256,7 +255,7 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         for (int b = 0; b < 2; ++b) mbar_init(bar(B_STG_FREE + b), 1);   // warp 4: copies have read block b
         mbar_init(bar(B_STG_READY), 4);              // the 4 epilogue warps staged their rows
         for (int sl = 0; sl < NSLOT_H; ++sl) mbar_init(bar(B_XDONE + sl), NXW);   // x_in warps done
-        for (int b = 0; b < NPASS; ++b) {
+        for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_LG_FULL + b), 1);       // owner: a pass of logits is complete
             mbar_init(bar(B_LG_EMPTY + b), 1);      // Sinkhorn warp: the pass is consumed
         }
@@ -529,8 +528,8 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
             }
             // [H_pre | res logits | post logits] of the owner's tokens -> the Sinkhorn ring;
             // a pass is BATCH / TPO tiles
-            const int kb = k % (BATCH / TPO), pb = k / (BATCH / TPO), b = pb % NPASS;
-            if (kb == 0 && !wait(bar(B_LG_EMPTY + b), ((pb / NPASS) & 1) ^ 1, E_LG_EMPTY)) break;
+            const int kb = k % (BATCH / TPO), pb = k / (BATCH / TPO), b = pb & 1;
+            if (kb == 0 && !wait(bar(B_LG_EMPTY + b), ((pb >> 1) & 1) ^ 1, E_LG_EMPTY)) break;
             if (lane < M) {
 #pragma unroll
                 for (int t = 0; t < TPO; ++t) ring[(b * BATCH + kb * TPO + t) * M + lane] = zt[t];
@@ -543,8 +542,8 @@ pre_tc_kernel(const __grid_constant__ Maps maps, const __nv_bfloat16* __restrict
         // (BATCH / TPO tiles of this owner) per pass
         const int npass = (my_tiles + BATCH / TPO - 1) / (BATCH / TPO);
         for (int pb = 0; pb < npass; ++pb) {
-            const int b = pb % NPASS;
-            if (!wait(bar(B_LG_FULL + b), (pb / NPASS) & 1, E_LG_FULL)) break;
+            const int b = pb & 1;
+            if (!wait(bar(B_LG_FULL + b), (pb >> 1) & 1, E_LG_FULL)) break;
             const int k = pb * (BATCH / TPO) + lane / TPO, t = lane % TPO;
             if (k < my_tiles) {
                 const float* L = ring + (b * BATCH + lane) * M;
