@@ -323,6 +323,7 @@ wide_proj_kernel(const __grid_constant__ WMaps maps, const uint8_t* __restrict__
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                 // packed phi and the scratch belong to the packing launch
 
     if (warp == 0) {
         // producer: stage g = (tile g / spt, atoms from al = (g % spt) * SW): one X box of
@@ -559,6 +560,7 @@ wide_xin_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ H
     const int per_tok = (chunks + 31) >> 5;
     const int64_t ntasks = Tn * per_tok;
     const int lane = threadIdx.x & 31;
+    pdl_wait();                 // H is the projection launch's
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t task = (((int64_t)blockIdx.x * blockDim.x) + threadIdx.x) >> 5; task < ntasks; task += nwarps) {
         const int64_t t = task / per_tok;
@@ -737,13 +739,17 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p) {
         cfg.blockDim = dim3(THREADS);
         cfg.dynamicSmemBytes = (size_t)p.smem;
         cfg.stream = a.stream;
-        cudaLaunchAttribute at[1];
+        cudaLaunchAttribute at[2];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = C;
         at[0].val.clusterDim.y = 1;
         at[0].val.clusterDim.z = 1;
+        // the set-up (barriers, TMEM) overlaps the packing launch's tail; pdl_wait precedes every
+        // access to the packed phi and the scratch
+        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, wide_proj_kernel<N>, maps, static_cast<const uint8_t*>(packed), scratch,
                                a.b_pre, a.b_post, a.b_res, a.a_pre, a.a_post, a.a_res, (int)a.T, a.d, a.eps,
                                a.t_max, a.H, a.h_out, ka_total, p.nstage, a.hc ? 1 : 0, g_wait_ns);
@@ -753,8 +759,10 @@ cudaError_t launch_n(const PreArgs& a, const Plan& p) {
         const int64_t per_tok = (a.d / 8 + 31) / 32;
         int64_t blocks = (a.T * per_tok * 32 + 255) / 256;
         if (blocks > (int64_t)di.sm_count * 8) blocks = (int64_t)di.sm_count * 8;
-        wide_xin_kernel<N><<<(unsigned)blocks, 256, 0, a.stream>>>(
-            static_cast<const __nv_bfloat16*>(a.X), a.H, a.T, a.d, static_cast<__nv_bfloat16*>(a.x_in));
+        e = launch_pdl(wide_xin_kernel<N>, dim3((unsigned)blocks), dim3(256), 0, a.stream,
+                       static_cast<const __nv_bfloat16*>(a.X), static_cast<const float*>(a.H), a.T, a.d,
+                       static_cast<__nv_bfloat16*>(a.x_in));
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
