@@ -49,8 +49,8 @@ NCU_TRAFFIC = {
     ("post", "bf16_T16384_n4_d4096_outliers"): (int((336.344832 + 210.074368) * 2e6), "e2d0eca830bf798b"),
     # the three launches of the two-pass path at T=4096: the projection and read-map kernels
     # scaled x2, the phi packing (no token dependence) once
-    ("pre", "bf16_T8192_n8_d4096"): (int(((279.602432 + 0.499200 + 268.970752 + 6.845440) * 2 + 10.491136) * 1e6),
-                                     "0dfa0d4015ab4244"),
+    ("pre", "bf16_T8192_n8_d4096"): (int(((279.610624 + 0.082176 + 268.969216 + 5.862144) * 2 + 10.491904) * 1e6),
+                                     "0811af1e75883c76"),
     # the six launches of one mhc_backward call at T=8192, scaled x2 (backward.cu + backward_tc.cu)
     ("backward", "bf16_T16384_n4_d4096_outliers"): (int((1286.790400 + 261.519104) * 2e6), "bab5f002ab08645e"),
 }
