@@ -98,6 +98,13 @@ def test_forward_host_validation(lib):
     assert lib.mhc_forward_host_workspace_bytes(ct, n, d, 5) == 0
     assert lib.mhc_forward_host_workspace_bytes(1 << 40, n, d, 1) == 0   # a chunk too large
 
+    def expect(ct, n, d, es):   # three sets of X, F_out, x_in, H, X_out, each 256-byte aligned
+        up = lambda b: (b + 255) // 256 * 256
+        m = n * n + 2 * n
+        return 3 * (2 * up(ct * n * d * es) + 2 * up(ct * d * es) + up(ct * m * 4))
+    for ct_, n_, d_, dt_, es in ((4, 4, 64, 1, 2), (1024, 4, 4096, 1, 2), (7, 3, 100, 0, 4), (1, 8, 8, 1, 2)):
+        assert lib.mhc_forward_host_workspace_bytes(ct_, n_, d_, dt_) == expect(ct_, n_, d_, es)
+
     W = A + 0x5000000                                # device workspace (256-aligned)
 
     def fh(Xh=A, Fh=A + 0x1000000, phi=A + 0x6000000, bp=A + 0x7000000, bq=A + 0x7000100,
